@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the TTT layer on B200.
+
+One step = one TTT-Linear full-batch layer forward (Gram pass, update, apply -- the whole
+path, one kernel) over one batch at the high-resolution stage-1 shape: B=32 images, a 56x56
+token grid (N=3136), one head of d=64, bf16 Q/K/V, fp32 W0, eta=1.  Inputs are seeded
+synthetic N(0,1)/sqrt(d) values.
+
+Timing: W warm-up steps, then EXACTLY K steps captured in one CUDA graph and timed with CUDA
+events on the launching stream, bracketed by a barrier and device synchronisation, max over
+ranks.  The steps cycle through R input/output sets whose total size exceeds four times the
+126 MB L2, so every step reads its inputs from HBM.  With --gpus N (torchrun) every rank runs
+its own batch (units are independent: weak scaling, no data-path collective).
+
+Extra keys: `roofline` (algorithmic bytes per launch / average launch time vs the measured
+HBM copy peak), `e2e` (same metric through the public API with pinned host buffers, copies
+inside the timed region), `cpu_baseline` (the fp64 oracle on the host cores, bounded
+sample), `clocks` (NVML samples during the timed region), `gpu_launches`, `other_paths`
+(device time of the conv, MLP and chunked paths at their shapes).
+
+`--impl reference` times the CPU oracle instead (the reference arm: there is no reference
+code to install; the oracle restates the method).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TTT-layer fwd tokens/s and achieved HBM GB/s (% of B200 peak) at N=3136"
+WL = dict(workload="ttt_linear_fullbatch", grid="56x56", B=32, H=1, N=3136, d=64, eta=1.0)
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e, cpu baseline, other paths")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops_sustained", 1364.1)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ rank plumbing ------
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def barrier(pg, device):
+    if pg is not None:
+        import torch
+        if device.type == "cuda":
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+def max_over_ranks(pg, x, device):
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks -------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every `period` s while active."""
+
+    def __init__(self, index, period=0.002):
+        self.samples = []
+        self.ok = False
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = statistics.median(s[0] for s in self.samples)
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = [n for b, n in REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ traffic record -----
+def kernel_traffic(kernel_files, summary_name):
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    h = hashlib.sha256()
+    for f in kernel_files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    path = os.path.join(ROOT, "profiles", summary_name)
+    try:
+        with open(path) as fh:
+            text = fh.read()
+    except OSError:
+        return None, sha
+    rec = {}
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            rec["traffic"] = float(line.split(":", 1)[1])
+        if line.startswith("kernel_source_sha:"):
+            rec["sha"] = line.split(":", 1)[1].strip()
+    if rec.get("sha") == sha and "traffic" in rec:
+        return rec["traffic"], sha
+    return None, sha
+
+
+# ------------------------------------------------------------------ CPU oracle ---------
+def cpu_oracle_rate(seconds, B, H, N, d, seed=0):
+    """Tokens/s of the fp64 oracle on the host cores for the bench workload (bounded)."""
+    import oracle
+    from linear_attention_split_b200 import inputs
+    inp = inputs.linear_inputs(B, H, N, d, dtype="bf16", seed=seed)
+    q, k, v, w0 = (oracle._f64(inp[x]) for x in ("q", "k", "v", "w0"))
+    threads = oracle.default_threads()
+    # one unit per thread per pass keeps every core busy; passes repeat until `seconds`
+    per = min(B, threads)
+    t0 = time.perf_counter()
+    tokens = 0
+    passes = 0
+    while True:
+        b0 = (passes * per) % B
+        sl = slice(b0, b0 + per)
+        oracle.linear_fullbatch(q[sl], k[sl], v[sl], w0, threads=threads)
+        tokens += q[sl].shape[0] * N
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{passes} passes of {per} units (b, h) x N={N} tokens each of the "
+                      f"B={B} batch, {dt:.1f} s wall, fp64 per-token loops, one unit per thread"}
+
+
+# ------------------------------------------------------------------ our arm ------------
+def run_ours(args):
+    import torch
+    from linear_attention_split_b200 import ttt
+
+    world, rank, local, pg = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_peak, tf_peak, peak_src = peaks()
+    B, H, N, d, eta = WL["B"], WL["H"], WL["N"], WL["d"], WL["eta"]
+    per_set = 4 * B * H * N * d * 2
+    R = max(2, math.ceil(4 * L2_BYTES / per_set))
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    sets = []
+    for _ in range(R):
+        q, k, v = (torch.randn((B, H, N, d), generator=g, device=dev) / math.sqrt(d) for _ in range(3))
+        sets.append(dict(q=q.bfloat16(), k=k.bfloat16(), v=v.bfloat16(),
+                         out=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)))
+    w0 = torch.randn((H, d, d), generator=g, device=dev) / math.sqrt(d)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        s = sets[i % R]
+        ttt.ttt_linear_fullbatch(s["q"], s["k"], s["v"], w0, s["out"], None, eta, None, stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            step(i)
+    torch.cuda.synchronize(dev)
+    assert ttt.device_error() == 0
+    # capture the K timed steps in one graph (launch overhead out of the measurement)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        graph.capture_begin()
+        for i in range(args.steps):
+            step(i)
+        graph.capture_end()
+    with torch.cuda.stream(stream):
+        graph.replay()  # graph upload and a warm replay (untimed)
+    torch.cuda.synchronize(dev)
+    launches0 = ttt.kernel_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(pg, ms, dev)
+    assert ttt.device_error() == 0
+    kernels_per_step = 1  # the tensor-core TTT-Linear path is a single kernel per call
+    gpu_launches = args.steps * kernels_per_step
+    ms_step = ms / args.steps
+    tokens_step = B * N
+    value = world * tokens_step * args.steps / (ms / 1e3)
+    alg_bytes = 8 * B * H * N * d
+    alg_flops = 6 * B * H * N * d * d
+    achieved = alg_bytes / (ms_step / 1e3) / 1e9
+    traffic, sha = kernel_traffic(["linear_attention_split_b200/csrc/linear_tc.cuh",
+                                   "linear_attention_split_b200/csrc/common.cuh"],
+                                  "linear_tc_56x56.md")
+    del graph
+
+    rec = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "TTT-Linear full-batch step, B=32 x 56x56 tokens (N=3136), 1 head, d=64, "
+                               "bf16 Q/K/V, fp32 W0, eta=1",
+                   "global_batch": B * world, "seq_len": N, "heads": H, "head_dim": d,
+                   "parallelism": f"independent batches per rank (dp{world}), no collective",
+                   "l2": f"{R} rotating input/output sets of {per_set / 1e6:.1f} MB "
+                         f"({R * per_set / 1e6:.0f} MB > 4x L2)",
+                   "timing": "K steps in one CUDA graph, CUDA events on the launching stream"},
+        "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "lintc::linear_tc_kernel<64>",
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "tensor_tflops": alg_flops / (ms_step / 1e3) / 1e12},
+        "gpu_launches": gpu_launches,
+        "library_launch_counter_delta": ttt.kernel_launch_count() - launches0,
+    }
+    rec["clocks"] = sampler.summary()
+
+    if not args.no_extras:
+        rec["e2e"] = e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, min(args.steps, 200), world, pg)
+        rec["other_paths"] = other_paths(ttt, dev, stream, hbm_peak, tf_peak)
+        if rank == 0 and world == 1:
+            rec["cpu_baseline"] = cpu_oracle_rate(args.cpu_seconds, B, H, N, d)
+        elif rank == 0:
+            rec["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(rec), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, steps, world, pg):
+    """Same metric through the public API with pinned host buffers: every step copies Q, K, V
+    host->device, runs the layer and reads O back to the host."""
+    import torch
+    g = torch.Generator()
+    g.manual_seed(7)
+    hq, hk, hv = (((torch.randn((B, H, N, d), generator=g) / math.sqrt(d)).bfloat16()).pin_memory()
+                  for _ in range(3))
+    ho = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv, do = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(4))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def one():
+        with torch.cuda.stream(stream):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            ttt.ttt_linear_fullbatch(dq, dk, dv, w0, do, None, eta, None, stream)
+            ho.copy_(do, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(pg, e0.elapsed_time(e1), dev)
+    nbytes = B * H * N * d * 2
+    return {"value": world * B * N * steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+            "ms_per_step": ms / steps, "steps": steps,
+            "note": "pinned host buffers, stream-ordered copies and the C-ABI call, eager launches"}
+
+
+def other_paths(ttt, dev, stream, hbm_peak, tf_peak):
+    """Device time per call of the other paths at their workload shapes (informational)."""
+    import torch
+    from linear_attention_split_b200 import inputs
+    res = {}
+
+    def timed(fn, iters):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(iters):
+                fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / iters
+
+    # 3x3 depthwise conv, B=32, 56x56, C=64
+    inp = {k: v.to(dev) for k, v in inputs.dwconv_inputs(32, 56, 56, 64).items()}
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(ttt.ttt_dwconv_fullbatch_workspace_bytes(32, 56, 56, 64, 1), dtype=torch.uint8,
+                     device=dev)
+    ms = timed(lambda: ttt.ttt_dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], out, None, 1.0,
+                                                ws, stream), 20)
+    nb = 8 * 32 * 3136 * 64
+    res["dwconv_56x56_c64"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
+                               "hbm_gbs": nb / (ms / 1e3) / 1e9, "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / hbm_peak,
+                               "note": "L2-resident inputs (51 MB), informational"}
+    # TTT-MLP, B=16, H=12, N=4096, d=64, h=256
+    inp = {k: v.to(dev) for k, v in inputs.mlp_inputs(16, 12, 4096, 64).items()}
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(ttt.ttt_mlp_fullbatch_workspace_bytes(16, 12, 4096, 64, 256, 1), dtype=torch.uint8,
+                     device=dev)
+    ms = timed(lambda: ttt.ttt_mlp_fullbatch(inp["q"], inp["k"], inp["v"], inp["w1"], inp["w2"], out, None,
+                                             None, 1.0, ws, stream), 5)
+    fl = 14 * 16 * 12 * 4096 * 64 * 256
+    res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3),
+                                 "tflops": fl / (ms / 1e3) / 1e12,
+                                 "frac_of_tensor_peak": fl / (ms / 1e3) / 1e12 / tf_peak}
+    # chunked bidirectional, B=8, H=3, N=6400, d=64, chunk 64
+    inp = {k: v.to(dev) for k, v in inputs.chunked_inputs(8, 3, 6400, 64).items()}
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(max(1, ttt.ttt_linear_chunked_bidir_workspace_bytes(8, 3, 6400, 64, 64, 1)),
+                     dtype=torch.uint8, device=dev)
+    ms = timed(lambda: ttt.ttt_linear_chunked_bidir(inp["q"], inp["k"], inp["v"], inp["w0"], out, 64, 1.0,
+                                                    ws, stream), 5)
+    res["chunked_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
+                                "us_per_chunk_step": ms * 1e3 / 100,
+                                "hbm_gbs_min_traffic": 8 * 8 * 3 * 6400 * 64 / (ms / 1e3) / 1e9}
+    assert ttt.device_error() == 0
+    return res
+
+
+# ------------------------------------------------------------------ reference arm ------
+def run_reference(args):
+    """The oracle as it stands, on the host cores, on this workload (bounded per-step sample)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from linear_attention_split_b200 import inputs
+    B, H, N, d, eta = WL["B"], WL["H"], WL["N"], WL["d"], WL["eta"]
+    threads = oracle.default_threads()
+    inp = inputs.linear_inputs(B, H, N, d, dtype="bf16", seed=0)
+    q, k, v, w0 = (oracle._f64(inp[x]) for x in ("q", "k", "v", "w0"))
+    # size each step so that warm-up + K steps stay within about two minutes
+    t0 = time.perf_counter()
+    oracle.linear_fullbatch(q[:1], k[:1], v[:1], w0, threads=1)
+    unit_s = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    units = max(1, min(B, threads, int(budget / max(unit_s, 1e-6) * min(threads, B))))
+    sl = slice(0, units)
+    for _ in range(args.warmup):
+        oracle.linear_fullbatch(q[sl], k[sl], v[sl], w0, eta, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear_fullbatch(q[sl], k[sl], v[sl], w0, eta, threads=threads)
+    dt = time.perf_counter() - t0
+    value = units * N * args.steps / dt
+    sample = (f"each step: {units} of the B={B} units (b, h) at N={N}, d={d}, fp64 oracle, "
+              f"{threads} threads")
+    rec = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": "TTT-Linear full-batch step, B=32 x 56x56 tokens (N=3136), 1 head, d=64, "
+                                  "bf16 Q/K/V, fp32 W0, eta=1", "global_batch": B, "seq_len": N,
+                      "parallelism": "host threads"},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(rec), flush=True)
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,131 @@
+/*
+ * ttt.h -- C ABI of the B200 (sm_100a) Test-Time-Training layer library, libttt_b200.so.
+ *
+ * The layer replaces attention by one step of inner training.  Per (batch b, head h) unit,
+ * with Q, K, V in R^{N x d} and an inner model F_W with initial weights W0, it forms
+ *     l(W) = (1/N) sum_i 1/2 ||F_W(k_i) - v_i||^2,     W* = W0 - eta * grad l(W0),
+ *     o_i  = F_{W*}(q_i).
+ * Source of the operation: "ViT^3: Unlocking Test-Time Training in Vision" (techloop.online
+ * blog post), section on rewriting attention as online learning (train F on (K, V), take
+ * W*, output F_{W*}(Q)) and its design-study section (single epoch, full batch, inner
+ * learning rate 1.0; no L1-type loss).  The squared loss with 1/N is this library's reading
+ * of a point the pages leave open.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers, dense row-major in the stated layout, and
+ *     16-byte aligned.  Q/K/V/out share one storage type `dtype` (TTT_F32 or TTT_BF16);
+ *     inner weights are always fp32.  Accumulation is fp32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
+ *     are asynchronous: they enqueue kernels and return; device-side faults surface at the
+ *     caller's next synchronisation.
+ *   - `workspace` is caller-owned device scratch of at least the size the matching
+ *     *_workspace_bytes() query returns for the same arguments (it may be NULL when that
+ *     size is 0).  The library allocates no device memory and keeps no per-call state.
+ *   - Arguments are checked on the host before anything is enqueued.  Return codes:
+ *       TTT_OK, TTT_ERR_INVALID_ARG (null pointer, size <= 0, misalignment, non-finite eta,
+ *       inconsistent shape), TTT_ERR_UNSUPPORTED (a size outside the supported range),
+ *       TTT_ERR_WORKSPACE (workspace too small), TTT_ERR_CUDA (a launch failed).
+ *   - Waits inside kernels are bounded; a wait that runs out sets a device error word that
+ *     ttt_device_error() reads (TTT_ERR_TIMEOUT).
+ *   - Optional outputs (w_star, ...) are fp32, exact before any bf16 rounding; pass NULL to
+ *     skip them.
+ */
+#ifndef TTT_B200_H
+#define TTT_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_INVALID_ARG = 1,
+    TTT_ERR_UNSUPPORTED = 2,
+    TTT_ERR_WORKSPACE = 3,
+    TTT_ERR_CUDA = 4,
+    TTT_ERR_TIMEOUT = 5
+} ttt_status;
+
+/* Static English text for a status code (never NULL). */
+const char* ttt_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int ttt_version(void);
+
+/* Number of kernels this library has enqueued since it was loaded (all devices, all
+ * threads).  Diagnostic: lets a caller count the device work behind a call. */
+unsigned long long ttt_kernel_launch_count(void);
+
+/* Reads and clears the device error word of the current device.  Synchronises the device.
+ * Writes the raw bits to *bits (may be NULL).  Returns TTT_OK when no kernel reported a
+ * problem, TTT_ERR_TIMEOUT when a bounded wait ran out, TTT_ERR_CUDA on a CUDA failure. */
+int ttt_device_error(unsigned int* bits);
+
+/* --------------------------------------------------------------------------------------
+ * TTT-Linear, full batch (F_W(x) = x W; TTT abstract of Sun et al.: "hidden state a linear
+ * model").  Per unit u = b*H + h:
+ *     G = K^T K, C = K^T V,  W* = W0[h] - (eta/N) (G W0[h] - C),  O = Q W*.
+ *   q, k, v, out : [B, H, N, d]   dtype
+ *   w0           : [H, d, d]      fp32, shared across the batch
+ *   w_star       : [B, H, d, d]   fp32 output, or NULL
+ * Supported: any N >= 1, B*H >= 1, 1 <= d <= 128; bf16 with d in {32, 64} runs the
+ * tensor-core kernel (one cluster per unit, no workspace), everything else the CUDA-core
+ * kernels (workspace needed).
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_fullbatch_workspace_bytes(int B, int H, int N, int d, int dtype);
+int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out,
+                         float* w_star, int B, int H, int N, int d, float eta, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * 3x3 depthwise-conv inner model on the Hg x Wg token grid (ViT^3 blog, design study: a
+ * 3x3 depthwise convolution as the visual inner module).  Per image b and channel c:
+ *     F_w(X)(y, x) = sum_{a,b in 0..2} w[a][b] X(y+a-1, x+b-1)   (zero padding, no bias)
+ *     g[a][b] = (1/N) sum_p r(p) K(p + (a-1, b-1)),  r = F_{w0}(K) - V,  N = Hg*Wg
+ *     w* = w0[c] - eta g,  O = F_{w*}(Q)
+ *   q, k, v, out : [B, Hg, Wg, C] channels-last (token index = row*Wg + col), dtype
+ *   w0           : [C, 3, 3] fp32, shared across the batch
+ *   w_star       : [B, C, 3, 3] fp32 output, or NULL
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_dwconv_fullbatch_workspace_bytes(int B, int Hg, int Wg, int C, int dtype);
+int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out,
+                         float* w_star, int B, int Hg, int Wg, int C, float eta, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * TTT-MLP, full batch (TTT abstract of Sun et al.: "hidden state a two-layer MLP"):
+ *     F(x) = gelu_tanh(x W1) W2,  gelu_tanh(u) = u/2 (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3)))
+ * with the gradient of l taken by hand (chain rule), one full-batch step, then O = F*(Q).
+ *   q, k, v, out : [B, H, N, d]   dtype
+ *   w1 : [H, d, hidden] fp32;  w2 : [H, hidden, d] fp32
+ *   w1_star : [B, H, d, hidden], w2_star : [B, H, hidden, d] fp32 outputs, or NULL
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_mlp_fullbatch_workspace_bytes(int B, int H, int N, int d, int hidden, int dtype);
+int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* w1,
+                      const float* w2, void* out, float* w1_star, float* w2_star, int B, int H,
+                      int N, int d, int hidden, float eta, int dtype, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * Chunked bidirectional TTT-Linear (Vision-TTT gist, "Technische samenvatting": update rule
+ * W_t = W_{t-1} - eta grad l(W_{t-1}; x_t), mini-batch gradient descent, forward and
+ * backward scan).  Per unit, with chunks c of `chunk` consecutive tokens (N % chunk == 0):
+ *     W <- W0[h];  for each chunk in order:  W <- W - (eta/chunk) K_c^T (K_c W - V_c);
+ *                                            O_c = Q_c W      (W after the chunk's update)
+ * run once in raster order and once in reverse raster order (both from W0); the layer
+ * output is the sum of the two scans, added in fp32 and rounded once.
+ *   q, k, v, out : [B, H, N, d] dtype;  w0 : [H, d, d] fp32
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int chunk, int dtype);
+int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const float* w0,
+                             void* out, int B, int H, int N, int d, int chunk, float eta,
+                             int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_B200_H */

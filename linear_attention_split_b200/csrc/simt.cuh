@@ -1,0 +1,308 @@
+// simt.cuh -- general CUDA-core kernels for every TTT path and both storage types.
+//
+// These serve the fp32 inputs (whose 1e-4 accuracy bar rules out bf16 tensor cores) and any
+// shape the tensor-core kernels do not cover.  One thread owns one output value and sums in
+// fp32 over the reduction axis, so the code follows the definition step by step:
+//   full-batch step  W* = W0 - eta * grad l(W0),  l(W) = (1/N) sum_i 1/2 ||F_W(k_i) - v_i||^2,
+//   then o_i = F_{W*}(q_i)  ("ViT^3" blog: attention rewritten as online learning, steps 1-3;
+//   single epoch, full batch, lr 1.0 per its inner-training study).
+// Every intermediate lives in the caller's workspace (fp32); the long sums over tokens are
+// accumulated in fp64, because the step W0 - eta*grad can cancel most of W0 (the 3x3 conv
+// model at eta = 1 keeps about 2% of it), which magnifies summation error in W*.
+#pragma once
+#include "common.cuh"
+
+namespace simt {
+
+constexpr int TPB = 256;
+
+// ------------------------------------------------------------------ TTT-Linear -------
+// gc[u][i][c] = sum_t k[u][t][i] * X[u][t][c'],  X = K for c < d, V for c >= d (c' = c mod d)
+template <typename T>
+__global__ void __launch_bounds__(TPB) linear_gram(const T* __restrict__ k, const T* __restrict__ v,
+                                                   float* __restrict__ gc, int N, int d) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    const int w2 = 2 * d;
+    if (e >= d * w2) return;
+    const int i = e / w2, c = e % w2;
+    const T* ku = k + u * N * d;
+    const T* xu = (c < d ? k : v) + u * N * d;
+    const int cc = c < d ? c : c - d;
+    double acc = 0.0;
+    for (int t = 0; t < N; ++t) acc = fma((double)to_f(ku[(long long)t * d + i]), (double)to_f(xu[(long long)t * d + cc]), acc);
+    gc[u * d * w2 + e] = (float)acc;
+}
+
+// W*[u] = W0[h] - (eta/N) (G W0[h] - C)
+__global__ void __launch_bounds__(TPB) linear_update(const float* __restrict__ gc, const float* __restrict__ w0,
+                                                     float* __restrict__ wst, float* __restrict__ w_star_out,
+                                                     int H, int d, float eta_over_n) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    if (e >= d * d) return;
+    const int i = e / d, j = e % d;
+    const float* G = gc + u * 2 * d * d + (long long)i * 2 * d;  // row i of [G | C]
+    const float* W0 = w0 + (u % H) * d * d;
+    float s = 0.f;
+    for (int m = 0; m < d; ++m) s = fmaf(G[m], W0[m * d + j], s);
+    const float w = W0[e] - eta_over_n * (s - G[d + j]);
+    wst[u * d * d + e] = w;
+    if (w_star_out) w_star_out[u * d * d + e] = w;
+}
+
+// out[u][t][j] = sum_m x[u][t][m] * W[u][m][j]
+template <typename T>
+__global__ void __launch_bounds__(TPB) linear_apply(const T* __restrict__ x, const float* __restrict__ w,
+                                                    T* __restrict__ out, int N, int d) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    if (e >= (long long)N * d) return;
+    const long long t = e / d;
+    const int j = (int)(e % d);
+    const float* W = w + u * d * d;
+    const T* xt = x + u * N * d + t * d;
+    float s = 0.f;
+    for (int m = 0; m < d; ++m) s = fmaf(to_f(xt[m]), W[m * d + j], s);
+    out[u * N * d + e] = from_f<T>(s);
+}
+
+// ------------------------------------------------------------------ 3x3 depthwise conv -
+// channels-last [B][Hg][Wg][C]; taps [C][3][3] (per image when per_image != 0: [B][C][3][3])
+template <typename T>
+__device__ __forceinline__ float dw_tap_sum(const T* img, const float* wc, int Hg, int Wg, int C, int y,
+                                            int x, int c) {
+    float s = 0.f;
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+        const int yy = y + a - 1;
+        if (yy < 0 || yy >= Hg) continue;
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            const int xx = x + b - 1;
+            if (xx < 0 || xx >= Wg) continue;
+            s = fmaf(wc[a * 3 + b], to_f(img[((long long)yy * Wg + xx) * C + c]), s);
+        }
+    }
+    return s;
+}
+
+// r[b][p][c] = conv_{w0}(K)(p, c) - V(p, c)
+template <typename T>
+__global__ void __launch_bounds__(TPB) dwconv_residual(const T* __restrict__ k, const T* __restrict__ v,
+                                                       const float* __restrict__ w0, float* __restrict__ r,
+                                                       int Hg, int Wg, int C) {
+    const long long b = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    const long long NC = (long long)Hg * Wg * C;
+    if (e >= NC) return;
+    const int c = (int)(e % C);
+    const long long p = e / C;
+    const int y = (int)(p / Wg), x = (int)(p % Wg);
+    r[b * NC + e] = dw_tap_sum(k + b * NC, w0 + c * 9, Hg, Wg, C, y, x, c) - to_f(v[b * NC + e]);
+}
+
+// w*[b][c][tap] = w0[c][tap] - (eta/N) sum_p r(p, c) K(p + offset(tap), c)
+template <typename T>
+__global__ void __launch_bounds__(TPB) dwconv_update(const T* __restrict__ k, const float* __restrict__ r,
+                                                     const float* __restrict__ w0, float* __restrict__ wst,
+                                                     float* __restrict__ w_star_out, int Hg, int Wg, int C,
+                                                     float eta_over_n) {
+    const long long b = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    if (e >= 9 * C) return;
+    const int tap = e / C, c = e % C;
+    const int da = tap / 3 - 1, db = tap % 3 - 1;
+    const long long NC = (long long)Hg * Wg * C;
+    const T* kb = k + b * NC;
+    const float* rb = r + b * NC;
+    double acc = 0.0;
+    for (int y = 0; y < Hg; ++y) {
+        const int yy = y + da;
+        if (yy < 0 || yy >= Hg) continue;
+        for (int x = 0; x < Wg; ++x) {
+            const int xx = x + db;
+            if (xx < 0 || xx >= Wg) continue;
+            acc = fma((double)rb[((long long)y * Wg + x) * C + c], (double)to_f(kb[((long long)yy * Wg + xx) * C + c]), acc);
+        }
+    }
+    const float w = (float)((double)w0[c * 9 + tap] - (double)eta_over_n * acc);
+    wst[(b * C + c) * 9 + tap] = w;
+    if (w_star_out) w_star_out[(b * C + c) * 9 + tap] = w;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(TPB) dwconv_apply(const T* __restrict__ q, const float* __restrict__ wst,
+                                                    T* __restrict__ out, int Hg, int Wg, int C) {
+    const long long b = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    const long long NC = (long long)Hg * Wg * C;
+    if (e >= NC) return;
+    const int c = (int)(e % C);
+    const long long p = e / C;
+    const int y = (int)(p / Wg), x = (int)(p % Wg);
+    out[b * NC + e] = from_f<T>(dw_tap_sum(q + b * NC, wst + (b * C + c) * 9, Hg, Wg, C, y, x, c));
+}
+
+// ------------------------------------------------------------------ TTT-MLP ----------
+// a[u][t][m] = gelu(sum_i x[u][t][i] W1[i][m]); gp = gelu'(...) when gp != nullptr.
+// W1 is per head ([H][d][hd]) or per unit ([U][d][hd]) when per_unit != 0.
+template <typename T>
+__global__ void __launch_bounds__(TPB) mlp_hidden(const T* __restrict__ x, const float* __restrict__ w1,
+                                                  float* __restrict__ a, float* __restrict__ gp, int H, int N,
+                                                  int d, int hd, int per_unit) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    if (e >= (long long)N * hd) return;
+    const long long t = e / hd;
+    const int m = (int)(e % hd);
+    const float* W1 = w1 + (per_unit ? u : u % H) * d * hd;
+    const T* xt = x + u * N * d + t * d;
+    float z = 0.f;
+    for (int i = 0; i < d; ++i) z = fmaf(to_f(xt[i]), W1[i * hd + m], z);
+    float g;
+    a[u * N * hd + e] = gelu_tanh_f(z, gp ? &g : nullptr);
+    if (gp) gp[u * N * hd + e] = g;
+}
+
+// y[u][t][j] = sum_m a[u][t][m] W2[m][j]; APPLY: out = y, else r = y - v
+template <typename T, bool APPLY>
+__global__ void __launch_bounds__(TPB) mlp_out(const float* __restrict__ a, const float* __restrict__ w2,
+                                               const T* __restrict__ v, float* __restrict__ r, T* __restrict__ out,
+                                               int H, int N, int d, int hd, int per_unit) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    if (e >= (long long)N * d) return;
+    const long long t = e / d;
+    const int j = (int)(e % d);
+    const float* W2 = w2 + (per_unit ? u : u % H) * hd * d;
+    const float* at = a + u * N * hd + t * hd;
+    float s = 0.f;
+    for (int m = 0; m < hd; ++m) s = fmaf(at[m], W2[m * d + j], s);
+    if (APPLY)
+        out[u * N * d + e] = from_f<T>(s);
+    else
+        r[u * N * d + e] = s - to_f(v[u * N * d + e]);
+}
+
+// dz[u][t][m] = gelu'(z) * sum_j r[u][t][j] W2[h][m][j]   (written over gp)
+__global__ void __launch_bounds__(TPB) mlp_dz(const float* __restrict__ r, const float* __restrict__ w2,
+                                              float* __restrict__ gp_dz, int H, int N, int d, int hd) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    if (e >= (long long)N * hd) return;
+    const long long t = e / hd;
+    const int m = (int)(e % hd);
+    const float* W2 = w2 + (u % H) * hd * d + (long long)m * d;
+    const float* rt = r + u * N * d + t * d;
+    float s = 0.f;
+    for (int j = 0; j < d; ++j) s = fmaf(rt[j], W2[j], s);
+    gp_dz[u * N * hd + e] *= s;
+}
+
+// W1*[u][i][m] = W1[h][i][m] - (eta/N) sum_t k[t][i] dz[t][m]
+template <typename T>
+__global__ void __launch_bounds__(TPB) mlp_update_w1(const T* __restrict__ k, const float* __restrict__ dz,
+                                                     const float* __restrict__ w1, float* __restrict__ w1s,
+                                                     float* __restrict__ w1_out, int H, int N, int d, int hd,
+                                                     float eta_over_n) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    if (e >= d * hd) return;
+    const int i = e / hd, m = e % hd;
+    const T* ku = k + u * N * d;
+    const float* du = dz + u * N * hd;
+    double s = 0.0;
+    for (int t = 0; t < N; ++t) s = fma((double)to_f(ku[(long long)t * d + i]), (double)du[(long long)t * hd + m], s);
+    const float w = (float)((double)w1[(u % H) * d * hd + e] - (double)eta_over_n * s);
+    w1s[u * d * hd + e] = w;
+    if (w1_out) w1_out[u * d * hd + e] = w;
+}
+
+// W2*[u][m][j] = W2[h][m][j] - (eta/N) sum_t a[t][m] r[t][j]
+__global__ void __launch_bounds__(TPB) mlp_update_w2(const float* __restrict__ a, const float* __restrict__ r,
+                                                     const float* __restrict__ w2, float* __restrict__ w2s,
+                                                     float* __restrict__ w2_out, int H, int N, int d, int hd,
+                                                     float eta_over_n) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    if (e >= hd * d) return;
+    const int m = e / d, j = e % d;
+    const float* au = a + u * N * hd;
+    const float* ru = r + u * N * d;
+    double s = 0.0;
+    for (int t = 0; t < N; ++t) s = fma((double)au[(long long)t * hd + m], (double)ru[(long long)t * d + j], s);
+    const float w = (float)((double)w2[(u % H) * hd * d + e] - (double)eta_over_n * s);
+    w2s[u * hd * d + e] = w;
+    if (w2_out) w2_out[u * hd * d + e] = w;
+}
+
+// ------------------------------------------------------------------ chunked scan -----
+// One block per (unit, direction).  Shared memory: W [d][d], G [d][d], R [RB][d] (fp32).
+// Direction 0 visits chunks 0..nc-1, direction 1 visits them nc-1..0 (reverse raster);
+// the order of tokens inside a chunk does not change its sums.
+constexpr int CH_RB = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(TPB) chunked_scan(const T* __restrict__ q, const T* __restrict__ k,
+                                                    const T* __restrict__ v, const float* __restrict__ w0,
+                                                    float* __restrict__ opart, int H, int N, int d, int chunk,
+                                                    float eta_over_b) {
+    extern __shared__ float sm[];
+    float* W = sm;
+    float* G = W + d * d;
+    float* R = G + d * d;
+    const long long u = blockIdx.x;
+    const int dir = blockIdx.y;
+    const int dd = d * d;
+    const long long base = u * N * d;
+    float* op = opart + (long long)dir * gridDim.x * N * d + base;
+    for (int e = threadIdx.x; e < dd; e += TPB) W[e] = w0[(u % H) * dd + e];
+    __syncthreads();
+    const int nc = N / chunk;
+    for (int ci = 0; ci < nc; ++ci) {
+        const int c0 = (dir == 0 ? ci : nc - 1 - ci) * chunk;
+        for (int e = threadIdx.x; e < dd; e += TPB) G[e] = 0.f;
+        __syncthreads();
+        for (int s0 = 0; s0 < chunk; s0 += CH_RB) {
+            const int nr = min(CH_RB, chunk - s0);
+            // residuals with W before this chunk's update
+            for (int e = threadIdx.x; e < nr * d; e += TPB) {
+                const int tt = e / d, j = e % d;
+                const long long t = c0 + s0 + tt;
+                float f = 0.f;
+                for (int m = 0; m < d; ++m) f = fmaf(to_f(k[base + t * d + m]), W[m * d + j], f);
+                R[e] = f - to_f(v[base + t * d + j]);
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < dd; e += TPB) {
+                const int i = e / d, j = e % d;
+                float g = G[e];
+                for (int tt = 0; tt < nr; ++tt) g = fmaf(to_f(k[base + (long long)(c0 + s0 + tt) * d + i]), R[tt * d + j], g);
+                G[e] = g;
+            }
+            __syncthreads();
+        }
+        for (int e = threadIdx.x; e < dd; e += TPB) W[e] -= eta_over_b * G[e];
+        __syncthreads();
+        // outputs of the chunk with the updated W
+        for (int e = threadIdx.x; e < chunk * d; e += TPB) {
+            const int tt = e / d, j = e % d;
+            const long long t = c0 + tt;
+            float s = 0.f;
+            for (int m = 0; m < d; ++m) s = fmaf(to_f(q[base + t * d + m]), W[m * d + j], s);
+            op[t * d + j] = s;
+        }
+        __syncthreads();
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(TPB) chunked_combine(const float* __restrict__ opart, T* __restrict__ out,
+                                                       long long total) {
+    const long long e = (long long)blockIdx.x * TPB + threadIdx.x;
+    if (e >= total) return;
+    out[e] = from_f<T>(opart[e] + opart[total + e]);
+}
+
+}  // namespace simt

@@ -1,0 +1,411 @@
+// ttt_api.cu -- the C ABI of libttt_b200.so (declared in include/ttt.h).
+//
+// Host-side argument checks, workspace sizing, the choice between the tensor-core kernels
+// and the general CUDA-core kernels, TMA descriptor encoding and kernel launches.  This is
+// the library's only translation unit, so every kernel shares one device error word.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "ttt.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "linear_tc.cuh"
+
+namespace {
+
+std::atomic<unsigned long long> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int smem_per_sm = 0;
+    int smem_optin = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_lock;
+
+int current_device(DeviceInfo** info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTT_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_dev_lock);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return TTT_ERR_CUDA;
+        d.ready = true;
+    }
+    *info = &d;
+    return TTT_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launched(int n) {
+    g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+dim3 grid_units(long long units, long long elems) {
+    return dim3((unsigned)units, (unsigned)((elems + simt::TPB - 1) / simt::TPB));
+}
+bool grid_ok(long long units, long long elems) {
+    return units >= 1 && units <= 0x7fffffffLL && (elems + simt::TPB - 1) / simt::TPB <= 65535;
+}
+
+// ------------------------------------------------------------------ TMA descriptors ----
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor [U][N][d] viewed as 3-D (d fastest), box {d, box_rows, 1}
+bool tmap_bf16_3d(CUtensorMap* m, const void* base, int d, int N, int U, int box_rows,
+                  CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)U};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+    cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ TTT-Linear --------
+bool linear_uses_tc(int d, int dtype) { return dtype == TTT_BF16 && (d == 32 || d == 64); }
+
+template <typename T>
+int linear_simt(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B,
+                int H, int N, int d, float eta, void* ws, cudaStream_t st) {
+    const long long U = (long long)B * H;
+    if (!grid_ok(U, 2LL * d * d) || !grid_ok(U, (long long)N * d)) return TTT_ERR_UNSUPPORTED;
+    float* gc = static_cast<float*>(ws);
+    float* wst = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)U * 2 * d * d * 4));
+    const float eta_over_n = (float)((double)eta / (double)N);
+    simt::linear_gram<T><<<grid_units(U, 2LL * d * d), simt::TPB, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), gc, N, d);
+    simt::linear_update<<<grid_units(U, (long long)d * d), simt::TPB, 0, st>>>(gc, w0, wst, w_star, H, d,
+                                                                               eta_over_n);
+    simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(
+        static_cast<const T*>(q), wst, static_cast<T*>(out), N, d);
+    return launched(3);
+}
+
+template <int D>
+int linear_tc(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B,
+              int H, int N, float eta, cudaStream_t st) {
+    using C = lintc::Cfg<D>;
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const long long U = (long long)B * H;
+    if (U > 65535) return TTT_ERR_UNSUPPORTED;
+
+    // split each unit over S CTAs of one cluster so that the grid fills two CTAs per SM
+    int S = 1;
+    while (S < 8 && U * S < 2LL * dev->sms && (N + 2 * S - 1) / (2 * S) >= 16) S *= 2;
+    const int t_cta = (N + S - 1) / S;
+    const int tiles = (t_cta + lintc::TILE_ROWS - 1) / lintc::TILE_ROWS;
+    const int stages = (D == 64) ? 2 : 4;
+    static_assert(C::MIN_STAGES <= 2, "scratch must fit the ring");
+    const int budget = dev->smem_per_sm / 2 - 1024;  // two CTAs per SM
+    auto qbytes = [&](int qres, int tt) {
+        const int rows = ((qres * tt + 15) / 16) * 16;
+        return ((rows * C::ROWB + 1023) / 1024) * 1024;
+    };
+    auto fixed = [&](int qres) { return stages * C::SLOT_BYTES + 2 * C::WT_BYTES + 8 * (2 * stages + qres) + 1024; };
+    int TT = ((t_cta + tiles - 1) / tiles + 7) / 8 * 8;
+    int qres = tiles;
+    while (qres > 0 && fixed(qres) + qbytes(qres, TT) > budget) --qres;
+    if (qres < tiles) {  // some Q tiles stream through the ring: they need 16-row tiles
+        TT = ((t_cta + tiles - 1) / tiles + 15) / 16 * 16;
+        qres = tiles;
+        while (qres > 0 && fixed(qres) + qbytes(qres, TT) > budget) --qres;
+    }
+    lintc::Params p;
+    p.w0 = w0;
+    p.w_star = w_star;
+    p.H = H;
+    p.N = N;
+    p.TT = TT;
+    p.tiles = tiles;
+    p.T = TT * tiles;
+    p.q_res = qres;
+    p.stages = stages;
+    p.q_region_bytes = qbytes(qres, TT);
+    p.eta_over_n = (float)((double)eta / (double)N);
+    const lintc::Layout<D> L(p);
+    const int smem = (int)L.total + 1024;
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+
+    const CUtensorMapSwizzle sw = (D == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap tk, tv, tq, to;
+    if (!tmap_bf16_3d(&tk, k, D, N, (int)U, TT, sw) || !tmap_bf16_3d(&tv, v, D, N, (int)U, TT, sw) ||
+        !tmap_bf16_3d(&tq, q, D, N, (int)U, TT, sw) || !tmap_bf16_3d(&to, out, D, N, (int)U, 8, sw))
+        return TTT_ERR_CUDA;
+
+    auto kern = lintc::linear_tc_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess)
+        return TTT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, (unsigned)U, 1);
+    cfg.blockDim = dim3(lintc::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, to, p) != cudaSuccess) return TTT_ERR_CUDA;
+    return launched(1);
+}
+
+int check_common(const void* q, const void* k, const void* v, const void* out, int dtype, float eta) {
+    if (!q || !k || !v || !out) return TTT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TTT_ERR_INVALID_ARG;
+    if (dtype != TTT_F32 && dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (!std::isfinite(eta)) return TTT_ERR_INVALID_ARG;
+    return TTT_OK;
+}
+
+// ------------------------------------------------------------------ depthwise conv ----
+size_t dwconv_ws(int B, int Hg, int Wg, int C) {
+    return align256((size_t)B * Hg * Wg * C * 4) + align256((size_t)B * C * 9 * 4);
+}
+
+template <typename T>
+int dwconv_simt(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B,
+                int Hg, int Wg, int C, float eta, void* ws, cudaStream_t st) {
+    const long long NC = (long long)Hg * Wg * C;
+    if (!grid_ok(B, NC) || !grid_ok(B, 9LL * C)) return TTT_ERR_UNSUPPORTED;
+    float* r = static_cast<float*>(ws);
+    float* wst = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)B * NC * 4));
+    const float eta_over_n = (float)((double)eta / ((double)Hg * Wg));
+    simt::dwconv_residual<T><<<grid_units(B, NC), simt::TPB, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), w0, r, Hg, Wg, C);
+    simt::dwconv_update<T><<<grid_units(B, 9LL * C), simt::TPB, 0, st>>>(static_cast<const T*>(k), r, w0, wst,
+                                                                         w_star, Hg, Wg, C, eta_over_n);
+    simt::dwconv_apply<T><<<grid_units(B, NC), simt::TPB, 0, st>>>(static_cast<const T*>(q), wst,
+                                                                  static_cast<T*>(out), Hg, Wg, C);
+    return launched(3);
+}
+
+// ------------------------------------------------------------------ TTT-MLP -----------
+size_t mlp_ws(int B, int H, int N, int d, int hd) {
+    const size_t U = (size_t)B * H;
+    return 2 * align256(U * N * hd * 4) + align256(U * N * d * 4) + 2 * align256(U * d * hd * 4);
+}
+
+template <typename T>
+int mlp_simt(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
+             float* w1_star, float* w2_star, int B, int H, int N, int d, int hd, float eta, void* ws,
+             cudaStream_t st) {
+    const long long U = (long long)B * H;
+    if (!grid_ok(U, (long long)N * hd) || !grid_ok(U, (long long)N * d) || !grid_ok(U, (long long)d * hd))
+        return TTT_ERR_UNSUPPORTED;
+    char* w = static_cast<char*>(ws);
+    float* A = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * N * hd * 4);
+    float* GP = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * N * hd * 4);
+    float* R = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * N * d * 4);
+    float* W1s = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * d * hd * 4);
+    float* W2s = reinterpret_cast<float*>(w);
+    const float eta_over_n = (float)((double)eta / (double)N);
+    const T* qq = static_cast<const T*>(q);
+    const T* kk = static_cast<const T*>(k);
+    const T* vv = static_cast<const T*>(v);
+    simt::mlp_hidden<T><<<grid_units(U, (long long)N * hd), simt::TPB, 0, st>>>(kk, w1, A, GP, H, N, d, hd, 0);
+    simt::mlp_out<T, false><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(A, w2, vv, R, nullptr, H, N,
+                                                                                  d, hd, 0);
+    simt::mlp_dz<<<grid_units(U, (long long)N * hd), simt::TPB, 0, st>>>(R, w2, GP, H, N, d, hd);
+    simt::mlp_update_w1<T><<<grid_units(U, (long long)d * hd), simt::TPB, 0, st>>>(kk, GP, w1, W1s, w1_star, H, N,
+                                                                                  d, hd, eta_over_n);
+    simt::mlp_update_w2<<<grid_units(U, (long long)d * hd), simt::TPB, 0, st>>>(A, R, w2, W2s, w2_star, H, N, d,
+                                                                               hd, eta_over_n);
+    simt::mlp_hidden<T><<<grid_units(U, (long long)N * hd), simt::TPB, 0, st>>>(qq, W1s, A, nullptr, H, N, d, hd,
+                                                                               1);
+    simt::mlp_out<T, true><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(A, W2s, nullptr, nullptr,
+                                                                                 static_cast<T*>(out), H, N, d,
+                                                                                 hd, 1);
+    return launched(7);
+}
+
+// ------------------------------------------------------------------ chunked scan ------
+size_t chunked_ws(int B, int H, int N, int d) { return align256((size_t)2 * B * H * N * d * 4); }
+
+template <typename T>
+int chunked_simt(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
+                 int d, int chunk, float eta, void* ws, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const long long U = (long long)B * H;
+    const long long total = U * N * d;
+    if (U > 0x7fffffffLL || (total + simt::TPB - 1) / simt::TPB > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+    const int smem = (2 * d * d + simt::CH_RB * d) * 4;
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(simt::chunked_scan<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+        return TTT_ERR_CUDA;
+    float* op = static_cast<float*>(ws);
+    const float eta_over_b = (float)((double)eta / (double)chunk);
+    simt::chunked_scan<T><<<dim3((unsigned)U, 2), simt::TPB, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), w0, op, H, N, d, chunk,
+        eta_over_b);
+    simt::chunked_combine<T><<<(unsigned)((total + simt::TPB - 1) / simt::TPB), simt::TPB, 0, st>>>(
+        op, static_cast<T*>(out), total);
+    return launched(2);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI ==========
+extern "C" {
+
+const char* ttt_status_string(int status) {
+    switch (status) {
+        case TTT_OK: return "ok";
+        case TTT_ERR_INVALID_ARG: return "invalid argument";
+        case TTT_ERR_UNSUPPORTED: return "unsupported size";
+        case TTT_ERR_WORKSPACE: return "workspace too small";
+        case TTT_ERR_CUDA: return "CUDA error";
+        case TTT_ERR_TIMEOUT: return "a device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int ttt_version(void) { return 100; }
+
+unsigned long long ttt_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ttt_device_error(unsigned int* bits) {
+    unsigned int v = 0, zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return TTT_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_ttt_device_error, sizeof(v)) != cudaSuccess) return TTT_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_ttt_device_error, &zero, sizeof(zero)) != cudaSuccess) return TTT_ERR_CUDA;
+    if (bits) *bits = v;
+    if (v & (TTT_DEVERR_TIMEOUT_TMA | TTT_DEVERR_TIMEOUT_PEER)) return TTT_ERR_TIMEOUT;
+    return v ? TTT_ERR_CUDA : TTT_OK;
+}
+
+// ------------------------------------------------------------------ TTT-Linear --------
+size_t ttt_linear_fullbatch_workspace_bytes(int B, int H, int N, int d, int dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+    if (linear_uses_tc(d, dtype)) return 0;
+    const size_t U = (size_t)B * H;
+    return align256(U * 2 * d * d * 4) + align256(U * d * d * 4);
+}
+
+int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star,
+                         int B, int H, int N, int d, float eta, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w0 || !aligned16(w0) || (w_star && !aligned16(w_star))) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return TTT_ERR_INVALID_ARG;
+    if (d > 128) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_linear_fullbatch_workspace_bytes(B, H, N, d, dtype);
+    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == TTT_BF16) {
+        if (d == 64) return linear_tc<64>(q, k, v, w0, out, w_star, B, H, N, eta, st);
+        if (d == 32) return linear_tc<32>(q, k, v, w0, out, w_star, B, H, N, eta, st);
+        return linear_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
+    }
+    return linear_simt<float>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
+}
+
+// ------------------------------------------------------------------ depthwise conv ----
+size_t ttt_dwconv_fullbatch_workspace_bytes(int B, int Hg, int Wg, int C, int dtype) {
+    (void)dtype;
+    if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return 0;
+    return dwconv_ws(B, Hg, Wg, C);
+}
+
+int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star,
+                         int B, int Hg, int Wg, int C, float eta, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w0 || !aligned16(w0) || (w_star && !aligned16(w_star))) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return TTT_ERR_INVALID_ARG;
+    const size_t need = ttt_dwconv_fullbatch_workspace_bytes(B, Hg, Wg, C, dtype);
+    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == TTT_BF16)
+        return dwconv_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, Hg, Wg, C, eta, workspace, st);
+    return dwconv_simt<float>(q, k, v, w0, out, w_star, B, Hg, Wg, C, eta, workspace, st);
+}
+
+// ------------------------------------------------------------------ TTT-MLP -----------
+size_t ttt_mlp_fullbatch_workspace_bytes(int B, int H, int N, int d, int hidden, int dtype) {
+    (void)dtype;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || hidden <= 0) return 0;
+    return mlp_ws(B, H, N, d, hidden);
+}
+
+int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
+                      float* w1_star, float* w2_star, int B, int H, int N, int d, int hidden, float eta, int dtype,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w1 || !w2 || !aligned16(w1) || !aligned16(w2)) return TTT_ERR_INVALID_ARG;
+    if ((w1_star && !aligned16(w1_star)) || (w2_star && !aligned16(w2_star))) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || hidden <= 0) return TTT_ERR_INVALID_ARG;
+    if (d > 256 || hidden > 4096) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_mlp_fullbatch_workspace_bytes(B, H, N, d, hidden, dtype);
+    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == TTT_BF16)
+        return mlp_simt<__nv_bfloat16>(q, k, v, w1, w2, out, w1_star, w2_star, B, H, N, d, hidden, eta, workspace,
+                                       st);
+    return mlp_simt<float>(q, k, v, w1, w2, out, w1_star, w2_star, B, H, N, d, hidden, eta, workspace, st);
+}
+
+// ------------------------------------------------------------------ chunked scan ------
+size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int chunk, int dtype) {
+    (void)dtype;
+    (void)chunk;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+    return chunked_ws(B, H, N, d);
+}
+
+int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const float* w0, void* out, int B,
+                             int H, int N, int d, int chunk, float eta, int dtype, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w0 || !aligned16(w0)) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0) return TTT_ERR_INVALID_ARG;
+    if (d > 128) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_linear_chunked_bidir_workspace_bytes(B, H, N, d, chunk, dtype);
+    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == TTT_BF16)
+        return chunked_simt<__nv_bfloat16>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
+    return chunked_simt<float>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
+}
+
+}  // extern "C"

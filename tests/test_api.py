@@ -1,0 +1,99 @@
+"""C ABI checks that need no GPU: the library loads, exports every function include/ttt.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+
+import pytest
+
+from linear_attention_split_b200 import build, ttt
+
+FAKE = ctypes.c_void_p(0x100000)      # 16-byte aligned, never dereferenced: checks fail first
+MISALIGNED = ctypes.c_void_p(0x100008)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ttt.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = ttt.declared_functions()
+    assert len(names) == 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.ttt_status_string(s)
+    assert L.ttt_status_string(99) == b"unknown status"
+    assert L.ttt_version() == 100
+
+
+def test_workspace_queries(L):
+    # tensor-core TTT-Linear needs no workspace; the CUDA-core paths do
+    assert L.ttt_linear_fullbatch_workspace_bytes(32, 1, 3136, 64, 1) == 0
+    assert L.ttt_linear_fullbatch_workspace_bytes(1, 1, 196, 64, 0) >= 3 * 64 * 64 * 4
+    assert L.ttt_linear_fullbatch_workspace_bytes(0, 1, 196, 64, 0) == 0
+    assert L.ttt_dwconv_fullbatch_workspace_bytes(2, 5, 5, 8, 1) > 0
+    assert L.ttt_mlp_fullbatch_workspace_bytes(1, 1, 10, 8, 32, 0) > 0
+    assert L.ttt_linear_chunked_bidir_workspace_bytes(1, 1, 64, 64, 16, 1) >= 0
+
+
+def lin(L, q=FAKE, w0=FAKE, B=1, H=1, N=16, d=64, eta=1.0, dt=1, ws=None, wsb=0):
+    return L.ttt_linear_fullbatch(q, FAKE, FAKE, w0, FAKE, None, B, H, N, d, eta, dt, ws, wsb, None)
+
+
+def test_linear_rejects_bad_arguments(L):
+    assert lin(L, q=None) == 1
+    assert lin(L, q=MISALIGNED) == 1
+    assert lin(L, w0=None) == 1
+    assert lin(L, B=0) == 1
+    assert lin(L, N=-3) == 1
+    assert lin(L, eta=float("nan")) == 1
+    assert lin(L, eta=float("inf")) == 1
+    assert lin(L, dt=7) == 1
+    assert lin(L, d=256) == 2
+    # the CUDA-core path needs a workspace
+    assert lin(L, dt=0) == 3
+    assert lin(L, dt=0, ws=FAKE, wsb=16) == 3
+
+
+def test_dwconv_rejects_bad_arguments(L):
+    f = L.ttt_dwconv_fullbatch
+    assert f(None, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 4, 8, 1.0, 1, FAKE, 1 << 20, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 0, 4, 8, 1.0, 1, FAKE, 1 << 20, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 1, 4, 4, 8, 1.0, 1, FAKE, 1 << 20, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 4, 8, float("nan"), 1, FAKE, 1 << 20, None) == 1
+
+
+def test_mlp_rejects_bad_arguments(L):
+    f = L.ttt_mlp_fullbatch
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 64, 64, 256, 1.0, 1, FAKE, 1 << 30, None]
+    a = list(args)
+    a[3] = None
+    assert f(*a) == 1
+    a = list(args)
+    a[12] = 0
+    assert f(*a) == 1
+    a = list(args)
+    a[11] = 512
+    assert f(*a) == 2
+    a = list(args)
+    a[16] = 8
+    assert f(*a) == 3
+
+
+def test_chunked_rejects_bad_arguments(L):
+    f = L.ttt_linear_chunked_bidir
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 100, 64, 64, 1.0, 1, FAKE, 1 << 30, None) == 1  # N % b
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, 1.0, 1, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, FAKE, FAKE, None, FAKE, 1, 1, 128, 64, 64, 1.0, 1, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 256, 64, 1.0, 1, FAKE, 1 << 30, None) == 2
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 4, 8)
+    with pytest.raises(ValueError):
+        ttt.ttt_linear_fullbatch(q, q, q, torch.zeros(1, 8, 8), q)

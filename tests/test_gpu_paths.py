@@ -1,0 +1,128 @@
+"""GPU parity of the depthwise-conv, TTT-MLP and chunked bidirectional paths (C ABI vs oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_split_b200 import inputs, ttt
+from tolerance import assert_close
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def cuda(inp):
+    return {k: v.to(DEV) for k, v in inp.items()}
+
+
+# ============================================================== depthwise conv ========
+def check_dwconv(B, Hg, Wg, C, dtype, eta=1.0, seed=0):
+    inp = inputs.dwconv_inputs(B, Hg, Wg, C, dtype=dtype, seed=seed)
+    g = cuda(inp)
+    out, ws = ttt.dwconv_fullbatch(g["q"], g["k"], g["v"], g["w0"], eta=eta, with_w_star=True)
+    assert ttt.device_error() == 0
+    ro, rw = oracle.dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], eta=eta)
+    dt = inp["q"].dtype
+    assert_close(out, ro, dt, f"dwconv O {B}x{Hg}x{Wg}x{C} {dtype}")
+    assert_close(ws, rw, torch.float32 if dt == torch.float32 else dt, "dwconv w*")
+
+
+def test_dwconv_56x56_bf16_full():
+    """Stage-1 shape: B=32, 56x56 grid, C=64, bf16, every output."""
+    check_dwconv(32, 56, 56, 64, "bf16")
+
+
+@pytest.mark.parametrize("Hg,Wg", [(1, 1), (1, 7), (7, 1), (3, 5), (14, 14), (17, 9)])
+def test_dwconv_grids(Hg, Wg):
+    check_dwconv(2, Hg, Wg, 64, "bf16", seed=Hg * 100 + Wg)
+
+
+@pytest.mark.parametrize("C", [8, 24, 3])
+def test_dwconv_channels(C):
+    check_dwconv(3, 10, 12, C, "bf16")
+
+
+@pytest.mark.parametrize("eta", [0.0, 0.37, -0.5])
+def test_dwconv_eta(eta):
+    check_dwconv(2, 8, 8, 64, "bf16", eta=eta)
+
+
+def test_dwconv_f32():
+    check_dwconv(2, 14, 14, 16, "f32")
+
+
+# ============================================================== TTT-MLP ===============
+def check_mlp(B, H, N, d, hidden, dtype, eta=1.0, seed=0, sample=None):
+    inp = inputs.mlp_inputs(B, H, N, d, hidden=hidden, dtype=dtype, seed=seed)
+    g = cuda(inp)
+    out, w1s, w2s = ttt.mlp_fullbatch(g["q"], g["k"], g["v"], g["w1"], g["w2"], eta=eta, with_w_star=True)
+    assert ttt.device_error() == 0
+    dt = inp["q"].dtype
+    wdt = torch.float32 if dt == torch.float32 else dt
+    units = [(b, h) for b in range(B) for h in range(H)] if sample is None else sample
+    for b, h in units:
+        ro, r1, r2 = oracle.mlp_fullbatch(inp["q"][b:b + 1, h:h + 1], inp["k"][b:b + 1, h:h + 1],
+                                          inp["v"][b:b + 1, h:h + 1], inp["w1"][h:h + 1],
+                                          inp["w2"][h:h + 1], eta=eta)
+        assert_close(out[b:b + 1, h:h + 1], ro, dt, f"mlp O unit ({b},{h})")
+        assert_close(w1s[b:b + 1, h:h + 1], r1, wdt, f"mlp W1* unit ({b},{h})")
+        assert_close(w2s[b:b + 1, h:h + 1], r2, wdt, f"mlp W2* unit ({b},{h})")
+
+
+def test_mlp_64x64_bf16_sampled():
+    """Full shape B=16, 12 heads, N=4096, d=64, hidden 256, compared on sampled units."""
+    check_mlp(16, 12, 4096, 64, 256, "bf16", sample=[(0, 0), (3, 7), (15, 11), (9, 4)])
+
+
+@pytest.mark.parametrize("N", [1, 100, 300, 1000])
+def test_mlp_small_full(N):
+    check_mlp(2, 2, N, 64, 256, "bf16", seed=N)
+
+
+@pytest.mark.parametrize("eta", [0.0, 0.37, -0.5])
+def test_mlp_eta(eta):
+    check_mlp(1, 2, 256, 64, 256, "bf16", eta=eta)
+
+
+def test_mlp_f32_and_other_widths():
+    check_mlp(2, 2, 64, 16, 64, "f32")
+    check_mlp(1, 2, 70, 32, 128, "bf16")
+
+
+# ============================================================== chunked bidirectional ==
+def check_chunked(B, H, N, d, chunk, dtype, eta=1.0, seed=0):
+    inp = inputs.chunked_inputs(B, H, N, d, dtype=dtype, seed=seed)
+    g = cuda(inp)
+    out = ttt.linear_chunked_bidir(g["q"], g["k"], g["v"], g["w0"], chunk, eta=eta)
+    assert ttt.device_error() == 0
+    ro = oracle.linear_chunked(inp["q"], inp["k"], inp["v"], inp["w0"], chunk, eta=eta, direction=0)
+    assert_close(out, ro, inp["q"].dtype, f"chunked B={B} H={H} N={N} b={chunk} {dtype}")
+    return out
+
+
+def test_chunked_80x80_bf16_full():
+    """1280^2 at patch 16: B=8, 3 heads of 64, N=6400, chunk 64, every output."""
+    check_chunked(8, 3, 6400, 64, 64, "bf16")
+
+
+@pytest.mark.parametrize("N,chunk", [(64, 64), (192, 64), (256, 16), (128, 32), (48, 1), (320, 320)])
+def test_chunked_shapes(N, chunk):
+    check_chunked(2, 2, N, 64, chunk, "bf16", seed=N + chunk)
+
+
+@pytest.mark.parametrize("eta", [0.0, 0.37, -0.5])
+def test_chunked_eta(eta):
+    check_chunked(1, 2, 512, 64, 64, "bf16", eta=eta)
+
+
+def test_chunked_f32():
+    check_chunked(2, 1, 96, 32, 16, "f32")
+
+
+def test_chunked_full_chunk_is_twice_fullbatch():
+    """chunk = N: each scan is the full-batch step, so the sum is twice the full-batch output."""
+    inp = inputs.linear_inputs(2, 2, 512, 64, dtype="bf16", seed=5)
+    g = cuda(inp)
+    out = ttt.linear_chunked_bidir(g["q"], g["k"], g["v"], g["w0"], 512)
+    ref, _ = oracle.linear_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"])
+    assert_close(out, 2 * ref, torch.bfloat16, "chunk = N")
