@@ -10,11 +10,13 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <algorithm>
 
 #include "ttt.h"
 #include "common.cuh"
 #include "simt.cuh"
 #include "linear_tc.cuh"
+#include "linear_tc5.cuh"
 
 namespace {
 
@@ -166,7 +168,8 @@ int linear_tc(const void* q, const void* k, const void* v, const float* w0, void
         return TTT_ERR_CUDA;
 
     auto kern = lintc::linear_tc_kernel<D>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return TTT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(S, (unsigned)U, 1);
@@ -181,6 +184,72 @@ int linear_tc(const void* q, const void* k, const void* v, const float* w0, void
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, to, p) != cudaSuccess) return TTT_ERR_CUDA;
+    return launched(1);
+}
+
+// d = 64: tcgen05 kernel (one cluster of S CTAs per unit, no workspace)
+int linear_tc5(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B, int H,
+               int N, float eta, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const long long U = (long long)B * H;
+    if (U > 65535) return TTT_ERR_UNSUPPORTED;
+    int S = 1;
+    while (S < 8 && U * S < 2LL * dev->sms && (N + 2 * S - 1) / (2 * S) >= 16) S *= 2;
+    const int t_cta = (N + S - 1) / S;
+    const int fixed = lin5::RING_BYTES + (int)sizeof(lin5::Bars) + 1024;
+    const int budget = dev->smem_per_sm / 2 - 1024;  // two CTAs per SM
+    const int qcap_rows = ((budget - fixed) / lin5::ROWB) / 8 * 8;
+    lin5::Params p;
+    const int tiles = (t_cta + lin5::TILE_ROWS - 1) / lin5::TILE_ROWS;
+    int TT = ((t_cta + tiles - 1) / tiles + 7) / 8 * 8;
+    if (TT * tiles <= qcap_rows && tiles <= lin5::MAX_QBOX) {
+        p.TT = TT;  // every Q row of the CTA stays resident
+        p.T = TT * tiles;
+        p.q_rows = p.T;
+    } else {        // Q streams in 128-token tiles after the first q_rows
+        p.TT = lin5::TILE_ROWS;
+        p.T = (t_cta + lin5::MT - 1) / lin5::MT * lin5::MT;
+        p.q_rows = std::min(p.T, qcap_rows / lin5::MT * lin5::MT);
+    }
+    p.q_region = (p.q_rows * lin5::ROWB + 1023) / 1024 * 1024;
+    // the last resident 128-row MMA tile may read past the Q rows: it must stay in the allocation
+    const int rows128 = (p.q_rows + lin5::MT - 1) / lin5::MT * lin5::MT;
+    if (rows128 * lin5::ROWB > p.q_region + lin5::RING_BYTES) return TTT_ERR_UNSUPPORTED;
+    if ((p.q_rows + p.TT - 1) / p.TT > lin5::MAX_QBOX) return TTT_ERR_UNSUPPORTED;
+    p.w0 = w0;
+    p.w_star = w_star;
+    p.H = H;
+    p.N = N;
+    p.eta_over_n = (float)((double)eta / (double)N);
+    int smem = p.q_region + fixed;
+    // at most two CTAs per SM: their two 256-column TMEM allocations fill the 512 columns
+    smem = std::max(smem, dev->smem_per_sm / 3 + 1024);
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+
+    CUtensorMap tk, tv, tq, tq128, to;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!tmap_bf16_3d(&tk, k, 64, N, (int)U, p.TT, sw) || !tmap_bf16_3d(&tv, v, 64, N, (int)U, p.TT, sw) ||
+        !tmap_bf16_3d(&tq, q, 64, N, (int)U, p.TT, sw) || !tmap_bf16_3d(&tq128, q, 64, N, (int)U, lin5::MT, sw) ||
+        !tmap_bf16_3d(&to, out, 64, N, (int)U, 8, sw))
+        return TTT_ERR_CUDA;
+    auto kern = lin5::linear_tc5_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+        return TTT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, (unsigned)U, 1);
+    cfg.blockDim = dim3(lin5::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, tq128, to, p) != cudaSuccess) return TTT_ERR_CUDA;
     return launched(1);
 }
 
@@ -333,7 +402,7 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == TTT_BF16) {
-        if (d == 64) return linear_tc<64>(q, k, v, w0, out, w_star, B, H, N, eta, st);
+        if (d == 64) return linear_tc5(q, k, v, w0, out, w_star, B, H, N, eta, st);
         if (d == 32) return linear_tc<32>(q, k, v, w0, out, w_star, B, H, N, eta, st);
         return linear_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
     }
