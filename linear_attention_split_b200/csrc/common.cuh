@@ -272,3 +272,24 @@ __device__ __forceinline__ void ld16(uint32_t taddr, float* v) {
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 }  // namespace tc
+
+// ----------------------------------------------------------------------- bulk DSMEM --
+// Copy `bytes` (multiple of 16) from this CTA's shared memory into CTA `rank` of the
+// cluster, at the same offset as `local_dst`; completion is counted on that CTA's barrier
+// at the same offset as `local_bar`.  (Plain bulk copy: no multicast.)
+__device__ __forceinline__ void bulk_push(const void* local_src, const void* local_dst, const uint64_t* local_bar,
+                                          uint32_t rank, uint32_t bytes) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dsmem_map(local_dst, rank)),
+        "r"(smem_u32(local_src)), "r"(bytes), "r"(dsmem_map(local_bar, rank))
+        : "memory");
+}
+
+// Prefetch a 3-D tile of a tensor into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
