@@ -17,6 +17,7 @@
 #include "simt.cuh"
 #include "linear_tc.cuh"
 #include "linear_tc5.cuh"
+#include "dwconv_fused.cuh"
 
 namespace {
 
@@ -272,6 +273,68 @@ size_t dwconv_ws(int B, int Hg, int Wg, int C) {
     return align256((size_t)B * Hg * Wg * C * 4) + align256((size_t)B * C * 9 * 4);
 }
 
+// bf16 [B][Hg][Wg][C] viewed as 4-D (channels fastest), box {C, Wg, 1, 1}, no swizzle
+bool tmap_bf16_rows(CUtensorMap* m, const void* base, int C, int Wg, int Hg, int B) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)Wg * C * 2, (cuuint64_t)Hg * Wg * C * 2};
+    cuuint32_t box[4] = {(cuuint32_t)C, (cuuint32_t)Wg, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool dwconv_fused_ok(int Hg, int Wg, int C, int dtype) {
+    return dtype == TTT_BF16 && C == dwc::C && Wg <= 64 && Hg <= 8 * dwc::MAX_R;
+}
+
+int dwconv_fused(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B,
+                 int Hg, int Wg, float eta, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    if (B > 65535) return TTT_ERR_UNSUPPORTED;
+    int S = 1;
+    while (S < 8 && S * 2 <= Hg) S *= 2;
+    dwc::Params p;
+    p.R = (Hg + S - 1) / S;
+    if (p.R > dwc::MAX_R) return TTT_ERR_UNSUPPORTED;
+    p.cw = (Wg + dwc::PXW - 1) / dwc::PXW;
+    p.slot_bytes = (dwc::PXW * p.cw + 2) * dwc::PXB;
+    p.nslots = std::max(dwc::KS + dwc::VS, p.R + 2);
+    p.w0 = w0;
+    p.w_star = w_star;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.Hg = Hg;
+    p.Wg = Wg;
+    p.eta_over_n = (float)((double)eta / ((double)Hg * Wg));
+    const int smem = p.nslots * p.slot_bytes + 2 * dwc::C * dwc::NTAP * 4 + (int)sizeof(dwc::Bars) + 128;
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    CUtensorMap tk, tv, tq;
+    if (!tmap_bf16_rows(&tk, k, dwc::C, Wg, Hg, B) || !tmap_bf16_rows(&tv, v, dwc::C, Wg, Hg, B) ||
+        !tmap_bf16_rows(&tq, q, dwc::C, Wg, Hg, B))
+        return TTT_ERR_CUDA;
+    auto kern = dwc::dwconv_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+        return TTT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, (unsigned)B, 1);
+    cfg.blockDim = dim3((p.cw + 1) * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, p) != cudaSuccess) return TTT_ERR_CUDA;
+    return launched(1);
+}
+
 template <typename T>
 int dwconv_simt(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B,
                 int Hg, int Wg, int C, float eta, void* ws, cudaStream_t st) {
@@ -417,8 +480,8 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
 
 // ------------------------------------------------------------------ depthwise conv ----
 size_t ttt_dwconv_fullbatch_workspace_bytes(int B, int Hg, int Wg, int C, int dtype) {
-    (void)dtype;
     if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return 0;
+    if (dwconv_fused_ok(Hg, Wg, C, dtype)) return 0;
     return dwconv_ws(B, Hg, Wg, C);
 }
 
@@ -431,6 +494,7 @@ int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const floa
     const size_t need = ttt_dwconv_fullbatch_workspace_bytes(B, Hg, Wg, C, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dwconv_fused_ok(Hg, Wg, C, dtype)) return dwconv_fused(q, k, v, w0, out, w_star, B, Hg, Wg, eta, st);
     if (dtype == TTT_BF16)
         return dwconv_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, Hg, Wg, C, eta, workspace, st);
     return dwconv_simt<float>(q, k, v, w0, out, w_star, B, Hg, Wg, C, eta, workspace, st);
