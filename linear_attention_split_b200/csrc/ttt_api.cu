@@ -18,6 +18,7 @@
 #include "linear_tc.cuh"
 #include "linear_tc5.cuh"
 #include "dwconv_fused.cuh"
+#include "chunked_tc.cuh"
 
 namespace {
 
@@ -398,6 +399,49 @@ int mlp_simt(const void* q, const void* k, const void* v, const float* w1, const
 // ------------------------------------------------------------------ chunked scan ------
 size_t chunked_ws(int B, int H, int N, int d) { return align256((size_t)2 * B * H * N * d * 4); }
 
+bool chunked_tc_ok(int B, int H, int d, int chunk, int dtype) {
+    return dtype == TTT_BF16 && d == chk::D && chunk == chk::CB && (long long)B * H <= 65535;
+}
+size_t chunked_tc_ws(int B, int H, int N) { return align256((size_t)B * H * N * chk::D * 4); }
+
+int chunked_tc(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
+               float eta, void* ws, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const int U = B * H;
+    chk::Params p;
+    p.w0 = w0;
+    p.park = static_cast<float*>(ws);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.H = H;
+    p.N = N;
+    p.nc = N / chk::CB;
+    p.eta_over_b = (float)((double)eta / (double)chk::CB);
+    const int smem = 2 * chk::STAGES * chk::STAGE + 2 * 2 * chk::WT + (int)sizeof(chk::Bars) + 1024;
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    CUtensorMap tk, tq, tv;
+    if (!tmap_bf16_3d(&tk, k, 64, N, U, chk::CB, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tmap_bf16_3d(&tq, q, 64, N, U, chk::CB, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TTT_ERR_CUDA;
+    {   // V: box of 16 columns x 64 tokens, no swizzle
+        auto fn = encode_fn();
+        if (!fn) return TTT_ERR_CUDA;
+        cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)U};
+        cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+        cuuint32_t box[3] = {chk::NCOL, chk::CB, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (fn(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(v), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return TTT_ERR_CUDA;
+    }
+    auto kern = chk::chunked_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return TTT_ERR_CUDA;
+    kern<<<dim3(chk::GROUPS, U), chk::THREADS, smem, st>>>(tk, tq, tv, p);
+    return launched(1);
+}
+
 template <typename T>
 int chunked_simt(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
                  int d, int chunk, float eta, void* ws, cudaStream_t st) {
@@ -526,9 +570,8 @@ int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* 
 
 // ------------------------------------------------------------------ chunked scan ------
 size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int chunk, int dtype) {
-    (void)dtype;
-    (void)chunk;
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+    if (chunked_tc_ok(B, H, d, chunk, dtype)) return chunked_tc_ws(B, H, N);
     return chunked_ws(B, H, N, d);
 }
 
@@ -542,6 +585,7 @@ int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const 
     const size_t need = ttt_linear_chunked_bidir_workspace_bytes(B, H, N, d, chunk, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (chunked_tc_ok(B, H, d, chunk, dtype)) return chunked_tc(q, k, v, w0, out, B, H, N, eta, workspace, st);
     if (dtype == TTT_BF16)
         return chunked_simt<__nv_bfloat16>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
     return chunked_simt<float>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
