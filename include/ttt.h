@@ -125,6 +125,30 @@ int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const 
                              void* out, int B, int H, int N, int d, int chunk, float eta,
                              int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
+/* --------------------------------------------------------------------------------------
+ * ttt_linear_chunked_bidir_noalloc -- the chunked bidirectional scan above, for callers that
+ * may not allocate device memory when they call (for example a runtime whose allocator is
+ * owned by someone else, code that must not trigger cudaMalloc's implicit device-wide
+ * synchronisation in a latency-critical loop, or an embedding that forbids allocation after
+ * start-up).  It takes no workspace: its scratch is a fixed 16 MiB array inside this
+ * library's device image, held by every device that loads the library until the process
+ * exits.  The pages have no counterpart to this entry point; it is a service of the library.
+ *   - Same arguments, layouts and results as ttt_linear_chunked_bidir, minus the workspace.
+ *   - Returns TTT_ERR_WORKSPACE when ttt_linear_chunked_bidir_workspace_bytes() for these
+ *     arguments exceeds ttt_linear_chunked_bidir_noalloc_max_bytes() (16 MiB: e.g. B*H*N up
+ *     to 65536 for bf16, d = chunk = 64); other errors as for the workspace version.
+ *   - Allocates nothing: no cudaMalloc/cudaFree or allocating library routine is called.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     for the current device; make that first call before any stream capture.
+ *   - Every call shares the one array and overwrites the parts it reads before reading them
+ *     (nothing needs to start at zero); calls that overlap on the GPU, on any streams of the
+ *     same device, race on it and must be serialised by the caller.
+ * ------------------------------------------------------------------------------------ */
+int ttt_linear_chunked_bidir_noalloc(const void* q, const void* k, const void* v, const float* w0,
+                                     void* out, int B, int H, int N, int d, int chunk, float eta,
+                                     int dtype, void* stream);
+size_t ttt_linear_chunked_bidir_noalloc_max_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -465,6 +465,29 @@ int chunked_simt(const void* q, const void* k, const void* v, const float* w0, v
     return launched(2);
 }
 
+// ------------------------------------------------------------------ no-allocation scan ---
+// Scratch for ttt_linear_chunked_bidir_noalloc: a fixed array in this library's device image,
+// so that callers who may not allocate device memory can still run the scan.  Each device
+// that loads the library holds it until the process exits.  Its device address is looked up
+// once per device (host code cannot use the symbol itself: on the host it names a stand-in).
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_scratch_addr[kMaxDevices];
+std::mutex g_noalloc_lock;
+
+int noalloc_scratch(void** addr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTT_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_noalloc_lock);
+    if (!g_noalloc_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return TTT_ERR_CUDA;
+        g_noalloc_scratch_addr[dev] = ptr;
+    }
+    *addr = g_noalloc_scratch_addr[dev];
+    return TTT_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI ==========
@@ -590,5 +613,18 @@ int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const 
         return chunked_simt<__nv_bfloat16>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
     return chunked_simt<float>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
 }
+
+// ------------------------------------------------------------------ no-allocation scan ---
+int ttt_linear_chunked_bidir_noalloc(const void* q, const void* k, const void* v, const float* w0, void* out,
+                                     int B, int H, int N, int d, int chunk, float eta, int dtype, void* stream) {
+    const size_t need = ttt_linear_chunked_bidir_workspace_bytes(B, H, N, d, chunk, dtype);
+    if (need > kNoAllocScratchBytes) return TTT_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (int rc = noalloc_scratch(&scratch)) return rc;
+    return ttt_linear_chunked_bidir(q, k, v, w0, out, B, H, N, d, chunk, eta, dtype, scratch, kNoAllocScratchBytes,
+                                    stream);
+}
+
+size_t ttt_linear_chunked_bidir_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 
 }  // extern "C"

@@ -67,6 +67,10 @@ def lib():
         L.ttt_linear_chunked_bidir_workspace_bytes.argtypes = [i, i, i, i, i, i]
         L.ttt_linear_chunked_bidir.restype = i
         L.ttt_linear_chunked_bidir.argtypes = [p, p, p, p, p, i, i, i, i, i, f, i, p, sz, p]
+        L.ttt_linear_chunked_bidir_noalloc.restype = i
+        L.ttt_linear_chunked_bidir_noalloc.argtypes = [p, p, p, p, p, i, i, i, i, i, f, i, p]
+        L.ttt_linear_chunked_bidir_noalloc_max_bytes.restype = sz
+        L.ttt_linear_chunked_bidir_noalloc_max_bytes.argtypes = []
         _lib = L
     return _lib
 
@@ -192,6 +196,20 @@ def ttt_linear_chunked_bidir(q, k, v, w0, out, chunk, eta=1.0, workspace=None, s
     rc = lib().ttt_linear_chunked_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(out), B, H, N, d,
                                         int(chunk), float(eta), dt, _ptr(ws), nbytes, _stream(stream))
     _check("ttt_linear_chunked_bidir", rc)
+    return out
+
+
+def ttt_linear_chunked_bidir_noalloc(q, k, v, w0, out, chunk, eta=1.0, stream=None):
+    """The chunked scan without a workspace argument: for callers that may not allocate
+    device memory at call time.  Its scratch is a fixed array inside the library's device
+    image (ttt_linear_chunked_bidir_noalloc_max_bytes() long); calls that overlap on the GPU
+    race on it."""
+    dt = _dtype(q, k, v, out)
+    _weights(w0)
+    B, H, N, d = q.shape
+    rc = lib().ttt_linear_chunked_bidir_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(out), B, H, N, d,
+                                                int(chunk), float(eta), dt, _stream(stream))
+    _check("ttt_linear_chunked_bidir_noalloc", rc)
     return out
 
 

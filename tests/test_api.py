@@ -18,7 +18,7 @@ def L():
 
 def test_exports_every_declared_symbol(L):
     names = ttt.declared_functions()
-    assert len(names) == 12
+    assert len(names) == 14
     for n in names:
         assert hasattr(L, n), n
 
@@ -97,3 +97,11 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 4, 8)
     with pytest.raises(ValueError):
         ttt.ttt_linear_fullbatch(q, q, q, torch.zeros(1, 8, 8), q)
+
+
+def test_noalloc_scan_rejects_sizes_beyond_its_scratch(L):
+    """8 images x 3 heads x 6400 tokens need 39 MB of scratch, more than the fixed 16 MiB:
+    rejected on the host with TTT_ERR_WORKSPACE before anything reaches the device."""
+    assert L.ttt_linear_chunked_bidir_noalloc_max_bytes() == 16 << 20
+    rc = L.ttt_linear_chunked_bidir_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 3, 6400, 64, 64, 1.0, 1, None)
+    assert rc == 3
