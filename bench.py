@@ -277,9 +277,9 @@ def run_ours(args):
     alg_bytes = 8 * B * H * N * d
     alg_flops = 6 * B * H * N * d * d
     achieved = alg_bytes / (ms_step / 1e3) / 1e9
-    traffic, sha = kernel_traffic(["linear_attention_split_b200/csrc/linear_tc.cuh",
+    traffic, sha = kernel_traffic(["linear_attention_split_b200/csrc/linear_tc5.cuh",
                                    "linear_attention_split_b200/csrc/common.cuh"],
-                                  "linear_tc_56x56.md")
+                                  "linear_tc5_56x56.md")
     del graph
 
     rec = {
@@ -297,7 +297,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": "lintc::linear_tc_kernel<64>",
+                     "kernel": "lin5::linear_tc5_kernel", "kernel_source_sha": sha,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor_tflops": alg_flops / (ms_step / 1e3) / 1e12},
         "gpu_launches": gpu_launches,
