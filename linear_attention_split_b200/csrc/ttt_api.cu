@@ -19,6 +19,7 @@
 #include "linear_tc5.cuh"
 #include "dwconv_fused.cuh"
 #include "chunked_tc.cuh"
+#include "mlp_tc.cuh"
 
 namespace {
 
@@ -396,6 +397,89 @@ int mlp_simt(const void* q, const void* k, const void* v, const float* w1, const
     return launched(7);
 }
 
+// tcgen05 TTT-MLP (bf16, d = 64, hidden = 256): grad -> update -> apply
+bool mlp_tc_ok(int B, int H, int d, int hidden, int dtype) {
+    return dtype == TTT_BF16 && d == mlp::D && hidden == mlp::HID && (long long)B * H <= 65535;
+}
+int mlp_splits(long long U, int N, int sms) {
+    // token splits per unit: fill whole waves of one CTA per SM, at least two tiles per CTA
+    int best = 1;
+    double best_eff = 0.0;
+    const int max_s = std::max(1, std::min(8, (N + 2 * mlp::MT - 1) / (2 * mlp::MT)));
+    for (int S = 1; S <= max_s; ++S) {
+        const long long ctas = U * S;
+        const long long waves = (ctas + sms - 1) / sms;
+        const double eff = (double)ctas / (double)(waves * sms);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = S;
+        }
+    }
+    return best;
+}
+size_t mlp_tc_ws(int B, int H, int N) {
+    DeviceInfo* dev = nullptr;
+    const int sms = current_device(&dev) == TTT_OK ? dev->sms : 148;
+    const long long U = (long long)B * H;
+    const int S = mlp_splits(U, N, sms);
+    return align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4) + 2 * align256((size_t)U * mlp::D * mlp::HID * 2);
+}
+
+int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
+           float* w1_star, float* w2_star, int B, int H, int N, float eta, void* ws, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const int U = B * H;
+    const int S = mlp_splits(U, N, dev->sms);
+    const int T = ((N + S - 1) / S + mlp::MT - 1) / mlp::MT * mlp::MT;
+    char* w = static_cast<char*>(ws);
+    float* part = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4);
+    __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(w);
+    w += align256((size_t)U * mlp::D * mlp::HID * 2);
+    __nv_bfloat16* w2b = reinterpret_cast<__nv_bfloat16*>(w);
+
+    CUtensorMap tk, tq, to;
+    if (!tmap_bf16_3d(&tk, k, 64, N, U, mlp::MT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tmap_bf16_3d(&tq, q, 64, N, U, mlp::MT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tmap_bf16_3d(&to, out, 64, N, U, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TTT_ERR_CUDA;
+    const int smem_g = 2 * mlp::WBYTES + 2 * mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::GradBars) + 1024;
+    const int smem_a = 2 * mlp::WBYTES + mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
+    if (smem_g > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(mlp::grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_g) != cudaSuccess ||
+        cudaFuncSetAttribute(mlp::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
+        return TTT_ERR_CUDA;
+    mlp::GradParams gp;
+    gp.w1 = w1;
+    gp.w2 = w2;
+    gp.v = static_cast<const __nv_bfloat16*>(v);
+    gp.part = part;
+    gp.H = H;
+    gp.N = N;
+    gp.T = T;
+    mlp::grad_kernel<<<dim3(S, U), mlp::THREADS, smem_g, st>>>(tk, gp);
+    mlp::UpdateParams up;
+    up.w1 = w1;
+    up.w2 = w2;
+    up.part = part;
+    up.w1_star = w1_star;
+    up.w2_star = w2_star;
+    up.w1b = w1b;
+    up.w2b = w2b;
+    up.H = H;
+    up.S = S;
+    up.eta_over_n = (float)((double)eta / (double)N);
+    mlp::update_kernel<<<dim3(U, 8), 256, 0, st>>>(up);
+    mlp::ApplyParams ap;
+    ap.w1b = w1b;
+    ap.w2b = w2b;
+    ap.N = N;
+    ap.T = T;
+    mlp::apply_kernel<<<dim3(S, U), mlp::THREADS, smem_a, st>>>(tq, to, ap);
+    return launched(3);
+}
+
 // ------------------------------------------------------------------ chunked scan ------
 size_t chunked_ws(int B, int H, int N, int d) { return align256((size_t)2 * B * H * N * d * 4); }
 
@@ -569,8 +653,8 @@ int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const floa
 
 // ------------------------------------------------------------------ TTT-MLP -----------
 size_t ttt_mlp_fullbatch_workspace_bytes(int B, int H, int N, int d, int hidden, int dtype) {
-    (void)dtype;
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || hidden <= 0) return 0;
+    if (mlp_tc_ok(B, H, d, hidden, dtype)) return mlp_tc_ws(B, H, N);
     return mlp_ws(B, H, N, d, hidden);
 }
 
@@ -585,6 +669,8 @@ int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* 
     const size_t need = ttt_mlp_fullbatch_workspace_bytes(B, H, N, d, hidden, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (mlp_tc_ok(B, H, d, hidden, dtype))
+        return mlp_tc(q, k, v, w1, w2, out, w1_star, w2_star, B, H, N, eta, workspace, st);
     if (dtype == TTT_BF16)
         return mlp_simt<__nv_bfloat16>(q, k, v, w1, w2, out, w1_star, w2_star, B, H, N, d, hidden, eta, workspace,
                                        st);
