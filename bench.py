@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, cpu baseline, other paths")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--only", choices=["dwconv", "mlp", "chunked"], default=None,
+                    help="time one other path alone (used for per-kernel ncu captures)")
     return ap.parse_args()
 
 
@@ -355,13 +357,15 @@ def e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, steps, world, pg):
             "note": "pinned host buffers, stream-ordered copies and the C-ABI call, eager launches"}
 
 
-def other_paths(ttt, dev, stream, hbm_peak, tf_peak):
-    """Device time per call of the other paths at their workload shapes (informational)."""
+def other_paths(ttt, dev, stream, hbm_peak, tf_peak, only=None, iters=None):
+    """Device time per call of the other paths at their workload shapes (informational).
+    `only` restricts the run to one path; `iters` overrides the timed call count."""
     import torch
     from linear_attention_split_b200 import inputs
     res = {}
 
-    def timed(fn, iters):
+    def timed(fn, n):
+        n = iters if iters is not None else n
         with torch.cuda.stream(stream):
             for _ in range(3):
                 fn()
@@ -369,46 +373,63 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_peak):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         with torch.cuda.stream(stream):
-            for _ in range(iters):
+            for _ in range(n):
                 fn()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / iters
+        return e0.elapsed_time(e1) / n
 
-    # 3x3 depthwise conv, B=32, 56x56, C=64
-    inp = {k: v.to(dev) for k, v in inputs.dwconv_inputs(32, 56, 56, 64).items()}
-    out = torch.empty_like(inp["q"])
-    ws = torch.empty(ttt.ttt_dwconv_fullbatch_workspace_bytes(32, 56, 56, 64, 1), dtype=torch.uint8,
-                     device=dev)
-    ms = timed(lambda: ttt.ttt_dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], out, None, 1.0,
-                                                ws, stream), 20)
-    nb = 8 * 32 * 3136 * 64
-    res["dwconv_56x56_c64"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
-                               "hbm_gbs": nb / (ms / 1e3) / 1e9, "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / hbm_peak,
-                               "note": "L2-resident inputs (51 MB), informational"}
-    # TTT-MLP, B=16, H=12, N=4096, d=64, h=256
-    inp = {k: v.to(dev) for k, v in inputs.mlp_inputs(16, 12, 4096, 64).items()}
-    out = torch.empty_like(inp["q"])
-    ws = torch.empty(ttt.ttt_mlp_fullbatch_workspace_bytes(16, 12, 4096, 64, 256, 1), dtype=torch.uint8,
-                     device=dev)
-    ms = timed(lambda: ttt.ttt_mlp_fullbatch(inp["q"], inp["k"], inp["v"], inp["w1"], inp["w2"], out, None,
-                                             None, 1.0, ws, stream), 5)
-    fl = 14 * 16 * 12 * 4096 * 64 * 256
-    res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3),
-                                 "tflops": fl / (ms / 1e3) / 1e12,
-                                 "frac_of_tensor_peak": fl / (ms / 1e3) / 1e12 / tf_peak}
-    # chunked bidirectional, B=8, H=3, N=6400, d=64, chunk 64
-    inp = {k: v.to(dev) for k, v in inputs.chunked_inputs(8, 3, 6400, 64).items()}
-    out = torch.empty_like(inp["q"])
-    ws = torch.empty(max(1, ttt.ttt_linear_chunked_bidir_workspace_bytes(8, 3, 6400, 64, 64, 1)),
-                     dtype=torch.uint8, device=dev)
-    ms = timed(lambda: ttt.ttt_linear_chunked_bidir(inp["q"], inp["k"], inp["v"], inp["w0"], out, 64, 1.0,
-                                                    ws, stream), 5)
-    res["chunked_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
-                                "us_per_chunk_step": ms * 1e3 / 100,
-                                "hbm_gbs_min_traffic": 8 * 8 * 3 * 6400 * 64 / (ms / 1e3) / 1e9}
+    def workspace(nbytes):
+        return torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
+
+    if only in (None, "dwconv"):  # 3x3 depthwise conv, B=32, 56x56, C=64
+        inp = {k: v.to(dev) for k, v in inputs.dwconv_inputs(32, 56, 56, 64).items()}
+        out = torch.empty_like(inp["q"])
+        ws = workspace(ttt.ttt_dwconv_fullbatch_workspace_bytes(32, 56, 56, 64, 1))
+        ms = timed(lambda: ttt.ttt_dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], out, None, 1.0,
+                                                    ws, stream), 20)
+        nb = 8 * 32 * 3136 * 64
+        res["dwconv_56x56_c64"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
+                                   "hbm_gbs": nb / (ms / 1e3) / 1e9,
+                                   "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / hbm_peak,
+                                   "note": "same inputs every call (51 MB, L2-resident), informational"}
+        del inp, out, ws
+    if only in (None, "mlp"):  # TTT-MLP, B=16, H=12, N=4096, d=64, h=256
+        inp = {k: v.to(dev) for k, v in inputs.mlp_inputs(16, 12, 4096, 64).items()}
+        out = torch.empty_like(inp["q"])
+        ws = workspace(ttt.ttt_mlp_fullbatch_workspace_bytes(16, 12, 4096, 64, 256, 1))
+        ms = timed(lambda: ttt.ttt_mlp_fullbatch(inp["q"], inp["k"], inp["v"], inp["w1"], inp["w2"], out, None,
+                                                 None, 1.0, ws, stream), 5)
+        fl = 14 * 16 * 12 * 4096 * 64 * 256
+        res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3),
+                                     "tflops": fl / (ms / 1e3) / 1e12,
+                                     "frac_of_tensor_peak": fl / (ms / 1e3) / 1e12 / tf_peak,
+                                     "peak": "sustained bf16 (MEASURED_PEAKS.json)"}
+        del inp, out, ws
+    if only in (None, "chunked"):  # chunked bidirectional, B=8, H=3, N=6400, d=64, chunk 64
+        inp = {k: v.to(dev) for k, v in inputs.chunked_inputs(8, 3, 6400, 64).items()}
+        out = torch.empty_like(inp["q"])
+        ws = workspace(ttt.ttt_linear_chunked_bidir_workspace_bytes(8, 3, 6400, 64, 64, 1))
+        ms = timed(lambda: ttt.ttt_linear_chunked_bidir(inp["q"], inp["k"], inp["v"], inp["w0"], out, 64, 1.0,
+                                                        ws, stream), 5)
+        res["chunked_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
+                                    "us_per_chunk_step": ms * 1e3 / 100,
+                                    "hbm_gbs_min_traffic": 8 * 8 * 3 * 6400 * 64 / (ms / 1e3) / 1e9}
+        del inp, out, ws
     assert ttt.device_error() == 0
     return res
+
+
+def run_only(args):
+    """One of the other paths alone (a small, self-contained command for ncu captures)."""
+    import torch
+    from linear_attention_split_b200 import ttt
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_peak, tf_peak, _ = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    res = other_paths(ttt, dev, stream, hbm_peak, tf_peak, only=args.only, iters=args.steps)
+    print(json.dumps({"only": args.only, "steps": args.steps, "result": res}), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm ------
@@ -458,6 +479,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_ours(args)
 
