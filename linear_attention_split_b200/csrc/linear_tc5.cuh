@@ -3,149 +3,195 @@
 //
 // Operation ("ViT^3" blog, online-learning rewrite of attention, steps 1-3; TTT-Linear of the
 // TTT abstract), per unit u = (batch b, head h) with Q, K, V in R^{N x 64}:
-//     G = K^T K,  C = K^T V,   W* = W0 - (eta/N) (G W0 - C),   O = Q W*
-// ((G W0 - C)/N is the full-batch gradient of (1/N) sum_i 1/2 ||k_i W - v_i||^2 at W0.)
+//     G = K^T K,  C = K^T V,   grad = G W0 - C,   W* = W0 - (eta/N) grad,   O = Q W*
+// (grad/N is the full-batch gradient of (1/N) sum_i 1/2 ||k_i W - v_i||^2 at W0.)
 //
-// Layout of the work (one thread-block cluster of S CTAs per unit, S in {1, 2, 4, 8}; CTA r
-// owns tokens [r*T, r*T + T); warp 0 = TMA producer, warp 1 = MMA issuer, warps 2-5 =
-// epilogue).  Shared memory is one pool used three ways in turn:
-//   1. Gram pass: the whole pool is a ring of 16 KB K/V slots (128-byte swizzle, plain TMA,
-//      no multicast); the issuer computes [G ; C^T] = [K | V]^T K with tcgen05.mma, M = 128
-//      (features of K then of V), N = 64, K-dim = tokens, both operands MN-major straight
-//      from the tiles, fp32 accumulator in tensor memory (TMEM).  Once the last K/V tile has
-//      landed the producer prefetches this CTA's Q rows into L2 (no shared memory needed).
-//   2. Reduction: the epilogue writes the partial as fp32 rows [G | C] (scratch).  After one
-//      cluster barrier each CTA pushes row block r' of its partial to CTA r' with bulk
-//      copies (completion counted on the receiver's mbarrier); CTA r adds the S blocks of
-//      rows [64r/S, 64(r+1)/S) in rank order (deterministic, no atomics), forms those rows of
-//      W* in fp32, stores them as bf16 hi + lo (hi = bf16(W*), lo = bf16(W* - hi)) in an
-//      MN-major block and pushes that block to every other CTA the same way.
-//   3. Apply: Q is copied from L2 into the region the received partials occupied, the issuer
-//      computes O = Q hi + Q lo per 128-token tile into four TMEM buffers, and the epilogue
-//      converts O to bf16 in place over Q and stores it with TMA (rows >= N are clipped).
-// If a CTA's Q rows do not fit the resident region, the rest stream through the scratch area
-// at the end.  A split cluster barrier (arrive once everything destined to a CTA has arrived,
-// wait before exit) keeps every pushed-from buffer alive until its copies are done.  Every
-// wait is bounded (common.cuh).
+// Work layout: one thread-block cluster of S CTAs per unit (S in {1, 2, 4, 8}), one CTA per
+// SM.  The unit's tokens are cut into tiles of TT <= 128 rows (TT a multiple of 16, chosen so
+// that every CTA gets the same number of tiles); CTA r takes tiles r, r + S, r + 2S, ...
+// Warp 0 = TMA producer, warp 1 = tcgen05 MMA issuer (one thread), warps 2-9 = epilogue
+// (warp w reads TMEM lane quarter w % 4, column half (w - 2) / 4).  The design keeps the
+// shared-memory traffic per HBM byte low: each K/V byte is written once by TMA and read once
+// or twice by the tensor cores.
+//
+//   1. Gram pass, per tile (V, K land in a ring slot by plain TMA, 128-byte swizzle):
+//        A += [V | K]^T K    tcgen05, M = 128 (features of V, then of K), N = 64, K-dim = the
+//                            TT token rows, both operands MN-major straight from the slot;
+//                            TMEM rows 0-63 hold this CTA's part of C^T, rows 64-127 of G.
+//      Once the ring is primed the remaining K/V tiles are requested into L2, so that HBM
+//      sees the whole stream at once.  Q is requested only once the Gram pass is done: it is
+//      not needed before the exchange below has finished, and it would slow K and V down.
+//   2. Partial gradient, transposed (G is symmetric):  grad^T = W0^T G - C^T.
+//      The epilogue writes this CTA's G as bf16 hi + lo (a K-major operand), the issuer
+//      computes D = W0_hi^T [G_hi | G_lo] (N = 128) and adds W0_lo^T G_hi to its first half
+//      (M = 128 MMAs whose rows >= 64 are not used), so that lane f holds D[f] and C^T[f] and
+//      D[f][0:64] + D[f][64:128] - C^T[f] is row f of this CTA's grad^T, with W0 and G kept to
+//      2^-17.
+//   3. Exchange: CTA c owns W* columns [c 64/S, (c+1) 64/S).  Every epilogue thread of lane
+//      quarters 0-1 sends its row half of D - C^T to the owner with st.async (completion
+//      counted on the owner's mbarrier); the owner adds the S contributions in rank order
+//      (deterministic, no atomics), forms W*^T rows = W0^T - (eta/N) grad^T in fp32 and sends
+//      them as bf16 hi + lo to every CTA of the cluster, again with st.async.
+//   4. Apply: Q tiles are loaded into the ring region, [O_hi | O_lo] = Q [W*_hi | W*_lo]
+//      (one N = 128 MMA chain per tile) into two TMEM buffers; the epilogue warps form two
+//      groups of four (one warp per lane quarter) that take alternate tiles: add the two
+//      halves, write O as bf16 over the consumed Q tile, one TMA store per tile (rows >= N
+//      are clipped by the hardware).
+// Every wait is bounded (common.cuh).  Launched with programmatic stream serialization: the
+// kernel waits for the previous grid before its first global access.
 #pragma once
 #include "common.cuh"
 
 namespace lin5 {
 
 constexpr int D = 64;
-constexpr int ROWB = 128;                 // bytes per token row (64 bf16)
-constexpr int THREADS = 192;              // producer, issuer, 4 epilogue warps
-constexpr int TILE_ROWS = 64;             // rows reserved per K or V tile in a ring slot
-constexpr int TILE_BYTES = TILE_ROWS * ROWB;
-constexpr int SLOT_BYTES = 2 * TILE_BYTES;  // K tile, V tile
-constexpr int MAX_SLOTS = 12;
-constexpr int SCR_LD = 2 * D;             // scratch row: G[i][0..63] | C[i][0..63], fp32
-constexpr int SCR_BYTES = D * SCR_LD * 4; // 32 KB
-constexpr int RECV_OFF = SCR_BYTES;       // received partial blocks, later the Q region
-constexpr int WG_BYTES = 2048;            // one 8-row group of W*: hi atom, then lo atom
-constexpr int W_BYTES = 8 * WG_BYTES;
-constexpr int MT = 128;                   // tokens per phase-2 MMA tile
-constexpr int TMEM_COLS = 256;            // phase-1 accumulator, then four phase-2 buffers
-constexpr int MAX_QBOX = 32;              // resident Q TMA boxes per CTA
-constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);
-constexpr uint32_t IDESC_APPLY = tc::idesc_bf16(128, 64, 0, 1);
+constexpr int ROWB = 128;                      // bytes per token row (64 bf16)
+constexpr int MT = 128;                        // rows reserved per tile (TT <= MT are used)
+constexpr int TILE_BYTES = MT * ROWB;          // 16 KB
+constexpr int SLOT_BYTES = 2 * TILE_BYTES;     // K, V
+constexpr int MAX_SLOTS = 6;
+constexpr int MAX_QT = 2 * MAX_SLOTS;          // Q tile buffers carved from the ring
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;   // producer, issuer, 8 epilogue warps
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int OP_BYTES = D * ROWB;             // one 64 x 64 bf16 K-major operand, 8 KB
+constexpr int RECV_BYTES = D * D * 4;          // S sources x (64/S) rows x 64 fp32 = 16 KB
+constexpr int FIXED_BYTES = 4 * OP_BYTES + RECV_BYTES;  // W0 hi/lo, W* hi/lo, receive area
+constexpr int TMEM_COLS = 512;
+constexpr int COL_A = 0;                       // Gram accumulator [C^T ; G]
+constexpr int COL_D = 64;                      // W0^T [G_hi | G_lo] (rows 0-63), 128 columns
+constexpr int COL_O = 256;                     // two [O_hi | O_lo] buffers of 128 columns
+constexpr int OBUFS = 2;
+constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
+constexpr uint32_t IDESC_WG = tc::idesc_bf16(128, 64, 0, 0);     // A K-major, B K-major
+constexpr uint32_t IDESC_WG2 = tc::idesc_bf16(128, 128, 0, 0);   // A K-major, B K-major, N = 128
+constexpr uint32_t IDESC_APPLY = tc::idesc_bf16(128, 128, 0, 0); // A K-major, B K-major
 
 struct Params {
-    const float* w0;   // [H][64][64]
-    float* w_star;     // [U][64][64] or nullptr
+    const float* w0;    // [H][64][64]
+    float* w_star;      // [U][64][64] or nullptr
     int H, N;
-    int T;             // tokens per CTA
-    int TT;            // tokens per K/V tile (multiple of 8, <= 64)
-    int q_rows;        // resident Q rows (multiple of 8; multiple of 128 when Q streams)
-    int w_off;         // byte offset of the W* block area in the pool
-    int slots;         // K/V ring slots during the Gram pass (pool / 16 KB)
+    int TT;             // token rows per tile (multiple of 16, <= 128)
+    int n_tiles;        // tiles per unit, ceil(N / TT)
+    int slots;          // ring slots (32 KB each)
+    int nq;             // Q tile buffers (16 KB each, carved from the ring)
     float eta_over_n;
 };
 
 struct Bars {
-    uint64_t full[MAX_SLOTS], empty[MAX_SLOTS], qfull[MAX_QBOX], gram_done, rfull, wfull, qgo, tfull[4],
-        tempty[4], sfull[2], sempty[2];
+    uint64_t full[MAX_SLOTS], empty[MAX_SLOTS], qfull[MAX_QT], qempty[MAX_QT], tfull[OBUFS], tempty[OBUFS],
+        w0ready, gram_done, gready, dfull, rfull, wfull, wlocal;
     uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-}
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ void wready_sync() { asm volatile("bar.sync 2, 160;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// scratch [64 rows][128 cols] fp32; float4 chunks XOR-swizzled by row to spread banks
-__device__ __forceinline__ int scr_idx(int r, int c) { return r * SCR_LD + ((((c >> 2) ^ (r & 31))) << 2) + (c & 3); }
-// W* element (i, j) of part p (0 = hi, 1 = lo): MN-major, 128-byte swizzled 8-row groups
-__device__ __forceinline__ uint32_t w_off(int i, int j, int p) {
-    return (i >> 3) * WG_BYTES + p * 1024 + swz<3>((i & 7) * ROWB + j * 2);
+// Bounded wait with cluster-scope acquire (data written by peer CTAs with st.async).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int err) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > TTT_SPIN_LIMIT_CYCLES) {
+            ttt_raise(err);
+            return false;
+        }
+    }
+}
+// 16 / 8 bytes into another CTA's shared memory, completion counted on its mbarrier.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     raddr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
+                 "r"(a), "r"(b), "r"(rbar)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+    return out;
+}
+// Byte offset of element (row n, column k) in a 64 x 64 bf16 K-major operand, 128-byte swizzle.
+__device__ __forceinline__ uint32_t op_off(int n, int k) {
+    return (uint32_t)(n >> 3) * 1024u + swz<3>((uint32_t)(n & 7) * ROWB + (uint32_t)k * 2u);
+}
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 1)
     linear_tc5_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q128,
-                      const __grid_constant__ CUtensorMap tm_o8, const __grid_constant__ CUtensorMap tm_o32,
+                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                       const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* pool = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* scr = reinterpret_cast<float*>(pool);
-    uint8_t* recv = pool + RECV_OFF;
-    uint8_t* qreg = pool + RECV_OFF;
-    uint8_t* wblk = pool + p.w_off;
-    Bars* bars = reinterpret_cast<Bars*>(pool + p.w_off + W_BYTES);
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* pool = base;                                   // ring slots, then Q tiles
+    uint8_t* fixed = base + p.slots * SLOT_BYTES;
+    uint8_t* w0op = fixed;                                  // [W0_hi^T ; W0_lo^T] (K-major, 128 rows)
+    uint8_t* wsop = fixed + 2 * OP_BYTES;                   // G hi, lo; later [W*_hi^T ; W*_lo^T]
+    float* recv = reinterpret_cast<float*>(fixed + 4 * OP_BYTES);
+    Bars* bars = reinterpret_cast<Bars*>(fixed + FIXED_BYTES);
 
     const uint32_t S = gridDim.x;  // one cluster spans the x dimension
     const uint32_t rank = cluster_ctarank();
     const int u = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = (int)rank * p.T;
-    const int n_valid = max(0, min(p.N - t0, p.T));
-    const int nkv = (n_valid + p.TT - 1) / p.TT;                   // K/V tiles with data
-    const int q_valid = min(n_valid, p.q_rows);                      // resident rows with data
-    const int nqbox = (q_valid + p.TT - 1) / p.TT;                   // resident Q boxes
-    const int n_res_mt = (q_valid + MT - 1) / MT;                    // resident 128-row tiles
-    const int n_mt = (n_valid + MT - 1) / MT;                        // all 128-row tiles
-    const int rp = D / (int)S;                                       // W* rows formed here
+    const int n_t = (int)rank < p.n_tiles ? (p.n_tiles - (int)rank + (int)S - 1) / (int)S : 0;  // tiles here
+    const int rp = D / (int)S;             // W* columns owned by each CTA
     const int r0 = (int)rank * rp;
-    const uint32_t pblk_bytes = (uint32_t)rp * SCR_LD * 4;           // one partial row block
-    const uint32_t wblk_bytes = (uint32_t)rp / 8 * WG_BYTES;         // one W* row block
+    const int NS = p.slots, NQ = p.nq, TT = p.TT;
 
     // ---- set-up ------------------------------------------------------------------------
     if (threadIdx.x == 0) {
-        for (int s = 0; s < p.slots; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        for (int j = 0; j < MAX_QBOX; ++j) mbar_init(&bars->qfull[j], 1);
+        for (int j = 0; j < NQ; ++j) {
+            mbar_init(&bars->qfull[j], 1);
+            mbar_init(&bars->qempty[j], 1);
+        }
+        for (int b = 0; b < OBUFS; ++b) {
+            mbar_init(&bars->tfull[b], 1);
+            mbar_init(&bars->tempty[b], EPI_WARPS / 2);
+        }
+        mbar_init(&bars->w0ready, EPI_WARPS);
         mbar_init(&bars->gram_done, 1);
+        mbar_init(&bars->gready, EPI_WARPS / 2);
+        mbar_init(&bars->dfull, 1);
         mbar_init(&bars->rfull, 1);
         mbar_init(&bars->wfull, 1);
-        mbar_init(&bars->qgo, 128);
-        for (int b = 0; b < 4; ++b) {
-            mbar_init(&bars->tfull[b], 1);
-            mbar_init(&bars->tempty[b], 4);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->sfull[b], 1);
-            mbar_init(&bars->sempty[b], 4);
-        }
+        mbar_init(&bars->wlocal, EPI_WARPS);
         mbar_fence_init();
-        // partial blocks and W* blocks of the S-1 other CTAs land here (bulk copies, in bytes)
-        mbar_expect_tx(&bars->rfull, (S - 1) * pblk_bytes);
-        mbar_expect_tx(&bars->wfull, (S - 1) * wblk_bytes);
-    }
-    if (p.TT < TILE_ROWS) {  // token rows [TT, 64) of every K/V tile: zero K-dim padding
-        const int pad16 = (TILE_ROWS - p.TT) * ROWB / 16;
-        for (int e = threadIdx.x; e < p.slots * 2 * pad16; e += THREADS) {
-            const int tile = e / pad16, w = e % pad16;
-            *reinterpret_cast<uint4*>(pool + tile * TILE_BYTES + p.TT * ROWB + w * 16) = make_uint4(0, 0, 0, 0);
-        }
+        // gradient rows and W* rows from the S - 1 other CTAs (st.async bytes)
+        mbar_expect_tx(&bars->rfull, (S - 1) * (uint32_t)rp * D * 4u);
+        mbar_expect_tx(&bars->wfull, (S - 1) * (uint32_t)rp * 2u * ROWB);
     }
     if (warp == 1) tc::alloc(&bars->tmem_base, TMEM_COLS);
-    fence_proxy_async_smem();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
+    cluster_arrive_release();  // this CTA's barriers exist: peers may signal them
+    griddep_wait();            // the previous grid on the stream has completed
     const uint32_t tmem = bars->tmem_base;
 
     if (warp == 0) {
@@ -154,293 +200,281 @@ __global__ void __launch_bounds__(THREADS, 2)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_q);
-            for (int i = 0; i < nkv; ++i) {
-                const int slot = i % p.slots, use = i / p.slots;
+            tma_prefetch_desc(&tm_o);
+            for (int i = 0; i < n_t; ++i) {
+                const int slot = i % NS, use = i / NS;
                 if (use > 0) mbar_wait(&bars->empty[slot], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 uint8_t* dst = pool + slot * SLOT_BYTES;
-                mbar_expect_tx(&bars->full[slot], 2 * p.TT * ROWB);
-                tma_load_3d(dst, &tm_k, 0, t0 + i * p.TT, u, &bars->full[slot]);
-                tma_load_3d(dst + TILE_BYTES, &tm_v, 0, t0 + i * p.TT, u, &bars->full[slot]);
-            }
-            // Q to L2 once the last K/V tile has landed: the Gram pass gets the bandwidth first
-            if (nkv > 0)
-                mbar_wait(&bars->full[(nkv - 1) % p.slots], ((nkv - 1) / p.slots) & 1, TTT_DEVERR_TIMEOUT_TMA);
-            for (int j = 0; j < nqbox; ++j) tma_prefetch_l2_3d(&tm_q, 0, t0 + j * p.TT, u);
-        }
-        __syncwarp();
-        cluster_sync_all();          // all Gram passes done: pools of every CTA may receive
-        if (lane == 0) {             // Q into shared memory once the received partials are summed
-            mbar_wait(&bars->qgo, 0, TTT_DEVERR_TIMEOUT_PEER);
-            fence_proxy_async_smem();
-            for (int j = 0; j < nqbox; ++j) {
-                mbar_expect_tx(&bars->qfull[j], p.TT * ROWB);
-                tma_load_3d(qreg + j * p.TT * ROWB, &tm_q, 0, t0 + j * p.TT, u, &bars->qfull[j]);
-            }
-        }
-        __syncwarp();
-        cluster_arrive_relaxed();
-        cluster_wait_acquire();      // every CTA received everything: scratch reusable
-        if (lane == 0 && n_mt > n_res_mt) {  // Q tiles beyond the resident region
-            fence_proxy_async_smem();
-            for (int t = n_res_mt; t < n_mt; ++t) {
-                const int k = t - n_res_mt, slot = k & 1, use = k >> 1;
-                if (use > 0) mbar_wait(&bars->sempty[slot], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
-                mbar_expect_tx(&bars->sfull[slot], MT * ROWB);
-                tma_load_3d(pool + slot * SLOT_BYTES, &tm_q128, 0, t0 + t * MT, u, &bars->sfull[slot]);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ================================ MMA issuer =====================================
-        if (lane == 0) {
-            for (int i = 0; i < nkv; ++i) {
-                const int slot = i % p.slots, use = i / p.slots;
-                mbar_wait(&bars->full[slot], use & 1, TTT_DEVERR_TIMEOUT_TMA);
-                tc::fence_after();
-                const uint32_t kb = smem_u32(pool + slot * SLOT_BYTES);
-                const int ks_n = (p.TT + 15) / 16;
-                for (int ks = 0; ks < ks_n; ++ks) {
-                    // A = [K | V]^T: MN-major, atoms K tile / V tile (LBO), 8-token groups (SBO)
-                    const uint64_t a = tc::smem_desc(kb + ks * 2048, TILE_BYTES, 1024, 2);
-                    const uint64_t b = tc::smem_desc(kb + ks * 2048, TILE_BYTES, 1024, 2);
-                    tc::mma_bf16(tmem, a, b, IDESC_GRAM, (i > 0 || ks > 0) ? 1 : 0);
-                }
-                tc::commit(&bars->empty[slot]);
-            }
-            if (nkv > 0) tc::commit(&bars->gram_done);
-        }
-        __syncwarp();
-        cluster_sync_all();
-        wready_sync();  // this CTA's own W* block is written
-        if (lane == 0) mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_PEER);  // and the peers' blocks
-        __syncwarp();
-        cluster_arrive_relaxed();
-        if (lane == 0 && n_mt > 0) {
-            tc::fence_after();
-            const uint32_t wb = smem_u32(wblk);
-            for (int t = 0; t < n_mt; ++t) {
-                const int buf = t & 3;
-                if (t >= 4) mbar_wait(&bars->tempty[buf], ((t >> 2) - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-                uint32_t ab;
-                if (t < n_res_mt) {
-                    const int r_lo = t * MT, r_hi = min(q_valid, r_lo + MT) - 1;
-                    for (int j = r_lo / p.TT; j <= r_hi / p.TT; ++j)
-                        mbar_wait(&bars->qfull[j], 0, TTT_DEVERR_TIMEOUT_TMA);
-                    ab = smem_u32(qreg) + t * MT * ROWB;
-                } else {
-                    const int k = t - n_res_mt;
-                    mbar_wait(&bars->sfull[k & 1], (k >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
-                    ab = smem_u32(pool) + (k & 1) * SLOT_BYTES;
-                }
-                tc::fence_after();
-                const uint32_t d = tmem + buf * 64;
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        // A = Q tile, K-major; B = W* (rows = K-dim), MN-major, 8-row groups 2 KB apart
-                        const uint64_t a = tc::smem_desc(ab + ks * 32, 16, 1024, 2);
-                        const uint64_t b = tc::smem_desc(wb + part * 1024 + ks * 2 * WG_BYTES, 16384, WG_BYTES, 2);
-                        tc::mma_bf16(d, a, b, IDESC_APPLY, (part | ks) ? 1 : 0);
+                const int row = ((int)rank + i * (int)S) * TT;
+                mbar_expect_tx(&bars->full[slot], 2 * TT * ROWB);
+                tma_load_3d(dst, &tm_v, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + TILE_BYTES, &tm_k, 0, row, u, &bars->full[slot]);
+                if (i == NS - 1)  // the rest of K and V into L2 now
+                    for (int j = NS; j < n_t; ++j) {
+                        tma_prefetch_l2_3d(&tm_k, 0, ((int)rank + j * (int)S) * TT, u);
+                        tma_prefetch_l2_3d(&tm_v, 0, ((int)rank + j * (int)S) * TT, u);
                     }
-                tc::commit(&bars->tfull[buf]);
+            }
+            // the ring is free once every Gram MMA has completed
+            if (n_t > 0) mbar_wait(&bars->gram_done, 0, TTT_DEVERR_TIMEOUT_TMA);
+            griddep_launch();
+            for (int t = 0; t < n_t; ++t) {
+                const int qs = t % NQ, use = t / NQ;
+                if (use > 0) mbar_wait(&bars->qempty[qs], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                mbar_expect_tx(&bars->qfull[qs], TT * ROWB);
+                tma_load_3d(pool + qs * TILE_BYTES, &tm_q, 0, ((int)rank + t * (int)S) * TT, u, &bars->qfull[qs]);
             }
         }
         __syncwarp();
         cluster_wait_acquire();
+        cluster_arrive_release();
+    } else if (warp == 1) {
+        // ================================ MMA issuer =====================================
+        if (lane == 0) {
+            // ---- Gram pass: A += [V | K]^T K per tile -------------------------------------
+            for (int i = 0; i < n_t; ++i) {
+                const int slot = i % NS;
+                mbar_wait(&bars->full[slot], (i / NS) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                const uint32_t vb = smem_u32(pool + slot * SLOT_BYTES);
+                for (int ks = 0; ks < TT / 16; ++ks)
+                    // A = [V | K]^T: MN-major, atoms V tile / K tile (LBO), 8-token groups (SBO)
+                    tc::mma_bf16(tmem + COL_A, tc::smem_desc(vb + ks * 2048, TILE_BYTES, 1024, 2),
+                                 tc::smem_desc(vb + TILE_BYTES + ks * 2048, TILE_BYTES, 1024, 2), IDESC_GRAM,
+                                 (i > 0 || ks > 0) ? 1 : 0);
+                tc::commit(&bars->empty[slot]);
+            }
+            if (n_t > 0) {
+                tc::commit(&bars->gram_done);
+                // ---- D = W0_hi^T [G_hi | G_lo], then D[:, 0:64] += W0_lo^T G_hi ----------------
+                // A rows 0-63 are W0_hi^T (or W0_lo^T); rows 64-127 read whatever operand follows
+                // in shared memory and land in D rows that are never read.
+                mbar_wait(&bars->w0ready, 0, TTT_DEVERR_TIMEOUT_PEER);
+                mbar_wait(&bars->gready, 0, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
+                const uint32_t wa = smem_u32(w0op), ga = smem_u32(wsop);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_D, tc::smem_desc(wa + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(ga + ks * 32, 16, 1024, 2), IDESC_WG2, ks > 0 ? 1 : 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_D, tc::smem_desc(wa + OP_BYTES + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(ga + ks * 32, 16, 1024, 2), IDESC_WG, 1);
+                tc::commit(&bars->dfull);
+            }
+
+            // ---- apply: [O_hi | O_lo] = Q [W*_hi | W*_lo] per tile -----------------------------
+            mbar_wait_cluster(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_PEER);   // the peers' W* rows
+            mbar_wait(&bars->wlocal, 0, TTT_DEVERR_TIMEOUT_PEER);          // and this CTA's own
+            fence_proxy_async_smem();  // W* rows were written by generic stores (local and st.async)
+            tc::fence_after();
+            const uint32_t wsa = smem_u32(wsop);
+            for (int t = 0; t < n_t; ++t) {
+                const int b = t % OBUFS, qs = t % NQ;
+                if (t >= OBUFS) mbar_wait(&bars->tempty[b], (t / OBUFS - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                const uint32_t qa = smem_u32(pool + qs * TILE_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_O + b * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(wsa + ks * 32, 16, 1024, 2), IDESC_APPLY, ks > 0 ? 1 : 0);
+                tc::commit(&bars->tfull[b]);
+            }
+        }
+        __syncwarp();
+        cluster_wait_acquire();
+        cluster_arrive_release();
     } else {
         // ================================ epilogue =======================================
-        const int q4 = warp & 3;              // TMEM lane quarter this warp may access
-        const int row = q4 * 32 + lane;       // accumulator row (lane) owned by this thread
-        const int et = threadIdx.x - 64;      // 0..127
-        const int jc = et & 63;               // W* column this thread forms
+        const int q4 = warp & 3;               // TMEM lane quarter this warp may access
+        const int h = (warp - 2) >> 2;         // column half
+        const int row = q4 * 32 + lane;        // tile row / accumulator lane of this thread
+        const int et = threadIdx.x - 64;       // 0..255
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         const float* W0 = p.w0 + (size_t)(u % p.H) * D * D;
 
-        // ---- partial of this CTA: TMEM -> scratch rows [G | C] -------------------------
+        // ---- W0^T as bf16 hi + lo, K-major (row = output feature f, k = input feature m) --
         {
-            float acc[64];
-            if (nkv > 0) {
-                mbar_wait(&bars->gram_done, 0, TTT_DEVERR_TIMEOUT_TMA);
-                tc::fence_after();
+            const int f = et & 63, mg = et >> 6;  // 16 input features per thread
+            uint32_t hi[8], lo[8];
 #pragma unroll
-                for (int c = 0; c < 64; c += 16) tc::ld16(tmem + ((uint32_t)(q4 * 32) << 16) + c, &acc[c]);
-                tc::wait_ld();
-            } else {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) acc[c] = 0.f;
-            }
-            fence_proxy_async_smem();  // the pool was last touched by TMA and the tensor cores
-            if (row < 64) {            // row `row` of G
-#pragma unroll
-                for (int c = 0; c < 64; c += 4)
-                    *reinterpret_cast<float4*>(&scr[scr_idx(row, c)]) =
-                        make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-            } else {                   // row j of C^T = column j of C
-                const int j = row - 64;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) scr[scr_idx(i, 64 + j)] = acc[i];
-            }
-        }
-        fence_proxy_async_smem();      // the scratch is read next by bulk copies
-        // column jc of W0, requested now so that the loads fly during the exchange below
-        float w0c[D], w0r[4];  // and W0[i][jc] for this thread's first four rows of W*
-#pragma unroll
-        for (int m = 0; m < D; ++m)
-            asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(w0c[m]) : "l"(W0 + m * D + jc));
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            asm volatile("ld.global.nc.f32 %0, [%1];"
-                         : "=f"(w0r[k])
-                         : "l"(W0 + min(r0 + (et >> 6) + 2 * k, D - 1) * D + jc));
-        tc::fence_before();
-        cluster_sync_all();            // every CTA of the cluster is past its Gram pass
-
-        // ---- reduce-scatter: push block r' to CTA r', then sum the blocks of rows r0.. -----
-        if (S > 1) {
-            if (et == 0) {
-                for (uint32_t k = 1; k < S; ++k) {
-                    const uint32_t dst = (rank + k) % S;
-                    // slot of this CTA in the receiver's area: (rank - dst - 1) mod S
-                    const uint32_t slot = (rank + S - dst - 1) % S;
-                    bulk_push(reinterpret_cast<const uint8_t*>(scr) + dst * pblk_bytes, recv + slot * pblk_bytes,
-                              &bars->rfull, dst, pblk_bytes);
-                }
-            }
-            mbar_wait(&bars->rfull, 0, TTT_DEVERR_TIMEOUT_PEER);
-            // the S blocks of rows r0.. in rank order; every block has the same in-block layout
-            const uint32_t scr_a = smem_u32(scr), recv_a = smem_u32(recv) - (uint32_t)r0 * SCR_LD * 4;
-            const int items = rp * (SCR_LD / 4);
-            for (int it = et; it < items; it += 128) {
-                const uint32_t off = (uint32_t)scr_idx(r0 + it / 32, (it % 32) * 4) * 4;
-                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (uint32_t q = 0; q < S; ++q) {
-                    const uint32_t slot = (q + S - rank - 1) % S;
-                    const uint32_t a = (q == rank) ? scr_a + off : recv_a + slot * pblk_bytes + off;
-                    float4 x;
-                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                 : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
-                                 : "r"(a));
-                    sum.x += x.x;
-                    sum.y += x.y;
-                    sum.z += x.z;
-                    sum.w += x.w;
-                }
-                *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(scr) + off) = sum;
-            }
-        }
-        fence_proxy_async_smem();      // the receive area is written next by TMA (Q)
-        mbar_arrive(&bars->qgo);
-        epi_sync();
-
-        // ---- W*[i][jc] = W0[i][jc] - (eta/N)(sum_m G[i][m] W0[m][jc] - C[i][jc]) -------------
-        // rows r0 + (et>>6) + 2k, four at a time with split accumulators (independent chains)
-        for (int i0 = r0 + (et >> 6); i0 < r0 + rp; i0 += 8) {
-            float w0i[4], cij[4], s0[4], s1[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = min(i0 + 2 * k, D - 1);
-                w0i[k] = (i0 == r0 + (et >> 6)) ? w0r[k] : __ldg(&W0[i * D + jc]);  // W0[i][jc]
-                cij[k] = scr[scr_idx(i, 64 + jc)];
-                s0[k] = 0.f;
-                s1[k] = 0.f;
+            for (int k = 0; k < 8; ++k) {
+                const int m = mg * 16 + 2 * k;
+                split_bf16(__ldg(&W0[m * D + f]), __ldg(&W0[(m + 1) * D + f]), hi[k], lo[k]);
             }
 #pragma unroll
-            for (int m = 0; m < D; m += 8) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int i = min(i0 + 2 * k, D - 1);
-                    const float4 g0 = *reinterpret_cast<const float4*>(&scr[scr_idx(i, m)]);
-                    const float4 g1 = *reinterpret_cast<const float4*>(&scr[scr_idx(i, m + 4)]);
-                    s0[k] = fmaf(g0.x, w0c[m], s0[k]);
-                    s1[k] = fmaf(g0.y, w0c[m + 1], s1[k]);
-                    s0[k] = fmaf(g0.z, w0c[m + 2], s0[k]);
-                    s1[k] = fmaf(g0.w, w0c[m + 3], s1[k]);
-                    s0[k] = fmaf(g1.x, w0c[m + 4], s0[k]);
-                    s1[k] = fmaf(g1.y, w0c[m + 5], s1[k]);
-                    s0[k] = fmaf(g1.z, w0c[m + 6], s0[k]);
-                    s1[k] = fmaf(g1.w, w0c[m + 7], s1[k]);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = i0 + 2 * k;
-                const float w = w0i[k] - p.eta_over_n * ((s0[k] + s1[k]) - cij[k]);
-                const float hi = __bfloat162float(__float2bfloat16_rn(w));
-                const float lo = w - hi;
-                const float hi_n = __shfl_xor_sync(0xffffffffu, hi, 1);
-                const float lo_n = __shfl_xor_sync(0xffffffffu, lo, 1);
-                if (i < r0 + rp) {
-                    if (p.w_star) p.w_star[(size_t)u * D * D + i * D + jc] = w;
-                    if ((jc & 1) == 0) {  // columns jc, jc+1 as one bf16 pair
-                        *reinterpret_cast<uint32_t*>(wblk + w_off(i, jc, 0)) = pack_bf16(hi, hi_n);
-                        *reinterpret_cast<uint32_t*>(wblk + w_off(i, jc, 1)) = pack_bf16(lo, lo_n);
-                    }
-                }
-            }
-        }
-        fence_proxy_async_smem();  // read next by the bulk copies and the tensor cores
-        wready_sync();
-        if (et == 0) {
-            const uint8_t* src = wblk + (r0 >> 3) * WG_BYTES;
-            for (uint32_t k = 1; k < S; ++k) bulk_push(src, src, &bars->wfull, (rank + k) % S, wblk_bytes);
-        }
-        cluster_arrive_relaxed();  // all partials destined here arrived and were consumed
-
-        // ---- O tiles: TMEM -> bf16 in place over Q -> TMA store; the next tile's accumulator
-        //      is read from TMEM while the current one is converted and stored
-        float o[64];
-        if (n_mt > 0) {
-            mbar_wait(&bars->tfull[0], 0, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
-#pragma unroll
-            for (int c = 0; c < 64; c += 16) tc::ld16(tmem + ((uint32_t)(q4 * 32) << 16) + c, &o[c]);
-            tc::wait_ld();
-        }
-        for (int t = 0; t < n_mt; ++t) {
-            const int buf = t & 3;
-            uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(o[2 * c], o[2 * c + 1]);
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->tempty[buf]);
-            if (t + 1 < n_mt) {  // start reading the next accumulator
-                const int nb = (t + 1) & 3;
-                mbar_wait(&bars->tfull[nb], ((t + 1) >> 2) & 1, TTT_DEVERR_TIMEOUT_PEER);
-                tc::fence_after();
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) tc::ld16(tmem + ((uint32_t)(q4 * 32) << 16) + nb * 64 + c, &o[c]);
-            }
-            const bool streamed = t >= n_res_mt;
-            uint8_t* tile = streamed ? pool + ((t - n_res_mt) & 1) * SLOT_BYTES : qreg + t * MT * ROWB;
-            const int tok = t * MT + row;  // token index inside this CTA
-            if (tok < n_valid) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(tile + swz<3>(row * ROWB + c * 16)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t off = op_off(f, mg * 16 + 8 * c);
+                *reinterpret_cast<uint4*>(w0op + off) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                *reinterpret_cast<uint4*>(w0op + OP_BYTES + off) =
+                    make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                const int r32 = q4 * 32;  // this warp's 32 rows of the tile
-                if (t * MT + r32 + 32 <= n_valid) {
-                    tma_store_3d(&tm_o32, 0, t0 + t * MT + r32, u, tile + r32 * ROWB);
-                } else {
-                    for (int k = 0; k < 4; ++k)
-                        if (t * MT + r32 + 8 * k < n_valid)
-                            tma_store_3d(&tm_o8, 0, t0 + t * MT + r32 + 8 * k, u, tile + (r32 + 8 * k) * ROWB);
+            if (lane == 0) mbar_arrive(&bars->w0ready);
+        }
+        // W0[4 cg + i][r0 + fl] for the W* entries this thread forms (up to four items)
+        const int items = rp * 16;
+        float w0o[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int it = et + k * EPI_THREADS;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w0o[k][i] = it < items ? __ldg(&W0[(4 * (it & 15) + i) * D + r0 + (it >> 4)]) : 0.f;
+        }
+
+        // ---- G rows of this CTA as bf16 hi + lo (a K-major operand; G is symmetric) -------
+        if (n_t > 0) {
+            mbar_wait(&bars->gram_done, 0, TTT_DEVERR_TIMEOUT_TMA);
+            tc::fence_after();
+            if (row >= D) {  // lane 64 + i holds G row i
+                float g[32];
+                tc::ld16(lane_base + COL_A + h * 32, &g[0]);
+                tc::ld16(lane_base + COL_A + h * 32 + 16, &g[16]);
+                tc::wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) split_bf16(g[8 * c + 2 * k], g[8 * c + 2 * k + 1], hi[k], lo[k]);
+                    const uint32_t off = op_off(row - D, h * 32 + 8 * c);
+                    *reinterpret_cast<uint4*>(wsop + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4*>(wsop + OP_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 }
-                tma_store_commit();
-                if (streamed) {
-                    tma_store_wait_read_all();
-                    mbar_arrive(&bars->sempty[(t - n_res_mt) & 1]);
+                fence_proxy_async_smem();  // read next by the tensor cores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->gready);
+            }
+        }
+
+        // ---- exchange: send this thread's row half of grad^T to the column owner -----------
+        cluster_wait_acquire();  // every CTA of the cluster has initialised its barriers
+        if (row < D) {
+            float x[32];
+            if (n_t > 0) {
+                float c[32], y[32];
+                mbar_wait(&bars->dfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                tc::ld16(lane_base + COL_D + h * 32, &x[0]);
+                tc::ld16(lane_base + COL_D + h * 32 + 16, &x[16]);
+                tc::ld16(lane_base + COL_D + 64 + h * 32, &y[0]);
+                tc::ld16(lane_base + COL_D + 64 + h * 32 + 16, &y[16]);
+                tc::ld16(lane_base + COL_A + h * 32, &c[0]);
+                tc::ld16(lane_base + COL_A + h * 32 + 16, &c[16]);
+                tc::wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) x[k] = (x[k] + y[k]) - c[k];
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) x[k] = 0.f;
+            }
+            const uint32_t owner = (uint32_t)(row / rp);  // row = W* column f
+            float* dst = recv + ((size_t)(rank * rp + row % rp) * D + h * 32);
+            if (owner == rank) {
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4*>(dst + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
+            } else {
+                const uint32_t ra = mapa_u32(smem_u32(dst), owner);
+                const uint32_t rb = mapa_u32(smem_u32(&bars->rfull), owner);
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    st_async_v4(ra + k * 4, rb, __float_as_uint(x[k]), __float_as_uint(x[k + 1]),
+                                __float_as_uint(x[k + 2]), __float_as_uint(x[k + 3]));
+            }
+        }
+        tc::fence_before();
+        epi_sync();  // this CTA's own contributions are in the receive area; D and G are read
+        mbar_wait_cluster(&bars->rfull, 0, TTT_DEVERR_TIMEOUT_PEER);
+
+        // ---- W*^T rows r0.. : sum the S contributions in rank order, then send ------------
+        {
+            const uint32_t wfull_peer_base = smem_u32(&bars->wfull);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = et + k * EPI_THREADS;
+                if (it < items) {
+                    const int fl = it >> 4, cg = it & 15;
+                    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (uint32_t src = 0; src < S; ++src) {
+                        const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)(src * rp + fl) * D + 4 * cg);
+                        s.x += v.x;
+                        s.y += v.y;
+                        s.z += v.z;
+                        s.w += v.w;
+                    }
+                    const int f = r0 + fl;
+                    const float w[4] = {w0o[k][0] - p.eta_over_n * s.x, w0o[k][1] - p.eta_over_n * s.y,
+                                        w0o[k][2] - p.eta_over_n * s.z, w0o[k][3] - p.eta_over_n * s.w};
+                    if (p.w_star) {
+                        float* ws = p.w_star + (size_t)u * D * D;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) ws[(4 * cg + i) * D + f] = w[i];
+                    }
+                    uint32_t hi0, lo0, hi1, lo1;
+                    split_bf16(w[0], w[1], hi0, lo0);
+                    split_bf16(w[2], w[3], hi1, lo1);
+                    const uint32_t off = op_off(f, 4 * cg);
+                    *reinterpret_cast<uint2*>(wsop + off) = make_uint2(hi0, hi1);
+                    *reinterpret_cast<uint2*>(wsop + OP_BYTES + off) = make_uint2(lo0, lo1);
+                    for (uint32_t kk = 1; kk < S; ++kk) {
+                        const uint32_t peer = (rank + kk) % S;
+                        const uint32_t rb = mapa_u32(wfull_peer_base, peer);
+                        st_async_v2(mapa_u32(smem_u32(wsop + off), peer), rb, hi0, hi1);
+                        st_async_v2(mapa_u32(smem_u32(wsop + OP_BYTES + off), peer), rb, lo0, lo1);
+                    }
                 }
             }
+            fence_proxy_async_smem();  // read next by the tensor cores
             __syncwarp();
-            if (t + 1 < n_mt) tc::wait_ld();
+            if (lane == 0) mbar_arrive(&bars->wlocal);
         }
-        if (lane == 0) tma_store_wait_all();
+        cluster_arrive_release();  // every remote store of this thread has been issued
+
+        // ---- O tiles: group h (one warp per lane quarter) takes tiles t = h, h + 2, ...:
+        //      TMEM -> (hi + lo) -> bf16 over the Q tile -> one TMA store per tile -------------
+        const bool storer = (q4 == 0 && lane == 0);
+        for (int t = h; t < n_t; t += 2) {
+            const int b = t % OBUFS, qs = t % NQ;
+            uint8_t* tile = pool + qs * TILE_BYTES;  // the MMA that read this Q tile has completed
+            mbar_wait(&bars->tfull[b], (t / OBUFS) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            tc::fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float oh[32], ol[32];
+                const uint32_t ob = lane_base + COL_O + b * 128 + half * 32;
+                tc::ld16(ob, &oh[0]);
+                tc::ld16(ob + 16, &oh[16]);
+                tc::ld16(ob + 64, &ol[0]);
+                tc::ld16(ob + 80, &ol[16]);
+                tc::wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(tile + swz<3>((uint32_t)row * ROWB + half * 64 + c * 16)) =
+                        make_uint4(pack_bf16(oh[8 * c] + ol[8 * c], oh[8 * c + 1] + ol[8 * c + 1]),
+                                   pack_bf16(oh[8 * c + 2] + ol[8 * c + 2], oh[8 * c + 3] + ol[8 * c + 3]),
+                                   pack_bf16(oh[8 * c + 4] + ol[8 * c + 4], oh[8 * c + 5] + ol[8 * c + 5]),
+                                   pack_bf16(oh[8 * c + 6] + ol[8 * c + 6], oh[8 * c + 7] + ol[8 * c + 7]));
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tempty[b]);
+            fence_proxy_async_smem();
+            group_sync(h);  // the group's 128 rows are written
+            if (storer) {
+                const int grow = ((int)rank + t * (int)S) * TT;  // rows >= N are clipped
+                tma_store_3d(&tm_o, 0, grow, u, tile);
+                tma_store_commit();
+                if (t + NQ < n_t) {  // the buffer is reloaded with a later Q tile
+                    tma_store_wait_read_all();
+                    mbar_arrive(&bars->qempty[qs]);
+                }
+            }
+        }
+        if (storer) tma_store_wait_all();
         cluster_wait_acquire();
     }
 

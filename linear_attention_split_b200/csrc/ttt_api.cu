@@ -190,57 +190,40 @@ int linear_tc(const void* q, const void* k, const void* v, const float* w0, void
     return launched(1);
 }
 
-// d = 64: tcgen05 kernel (one cluster of S CTAs per unit, no workspace)
+// d = 64: tcgen05 kernel (one cluster of S CTAs per unit, one CTA per SM, no workspace)
 int linear_tc5(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B, int H,
                int N, float eta, cudaStream_t st) {
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     const long long U = (long long)B * H;
     if (U > 65535) return TTT_ERR_UNSUPPORTED;
-    int S = 1;
-    while (S < 8 && U * S < 2LL * dev->sms && (N + 2 * S - 1) / (2 * S) >= 16) S *= 2;
-    const int t_cta = (N + S - 1) / S;
-    const int recv = (S - 1) * (64 / S) * lin5::SCR_LD * 4;   // partial blocks from the peers
-    const int extra = (int)sizeof(lin5::Bars) + 1024;          // barriers + alignment slack
-    const int budget = dev->smem_per_sm / 2 - 1024;             // two CTAs per SM
-    const int qcap_rows = (budget - lin5::SCR_BYTES - lin5::W_BYTES - extra) / lin5::ROWB / 8 * 8;
     lin5::Params p;
-    const int tiles = (t_cta + lin5::TILE_ROWS - 1) / lin5::TILE_ROWS;
-    const int TT = ((t_cta + tiles - 1) / tiles + 7) / 8 * 8;
-    if (TT * tiles <= qcap_rows && tiles <= lin5::MAX_QBOX) {
-        p.TT = TT;  // every Q row of the CTA stays resident
-        p.T = TT * tiles;
-        p.q_rows = p.T;
-    } else {        // Q streams in 128-token tiles after the first q_rows
-        p.TT = lin5::TILE_ROWS;
-        p.T = (t_cta + lin5::MT - 1) / lin5::MT * lin5::MT;
-        p.q_rows = std::min(p.T, qcap_rows / lin5::MT * lin5::MT);
-    }
-    if ((p.q_rows + p.TT - 1) / p.TT > lin5::MAX_QBOX) return TTT_ERR_UNSUPPORTED;
-    const int q_region = (p.q_rows * lin5::ROWB + 1023) / 1024 * 1024;
-    int w_off = lin5::RECV_OFF + std::max(q_region, recv);
-    // the last resident 128-row MMA tile may read past the Q rows: keep it inside the pool
-    const int rows128 = (p.q_rows + lin5::MT - 1) / lin5::MT * lin5::MT;
-    w_off = std::max(w_off, lin5::RECV_OFF + rows128 * lin5::ROWB - lin5::W_BYTES);
-    const int pool = w_off + lin5::W_BYTES;
-    p.w_off = w_off;
-    p.slots = std::min(lin5::MAX_SLOTS, pool / lin5::SLOT_BYTES);
+    // split each unit over S CTAs while the grid stays within one CTA per SM, then pick the
+    // tile height (multiple of 16, <= 128) that gives every CTA the same number of tiles
+    const int t128 = (N + lin5::MT - 1) / lin5::MT;
+    int S = 1;
+    while (S < 8 && U * S * 2 <= dev->sms && S * 2 <= t128) S *= 2;
+    const int per_cta = (N + S - 1) / S;
+    const int k_tiles = (per_cta + lin5::MT - 1) / lin5::MT;
+    p.TT = ((per_cta + k_tiles - 1) / k_tiles + 15) / 16 * 16;
+    p.n_tiles = (N + p.TT - 1) / p.TT;
+    const int extra = lin5::FIXED_BYTES + (int)sizeof(lin5::Bars) + 1024;  // + alignment slack
+    p.slots = std::min(lin5::MAX_SLOTS, (dev->smem_optin - extra) / lin5::SLOT_BYTES);
     if (p.slots < 2) return TTT_ERR_UNSUPPORTED;
+    p.nq = std::min(lin5::MAX_QT, p.slots * lin5::SLOT_BYTES / lin5::TILE_BYTES);
     p.w0 = w0;
     p.w_star = w_star;
     p.H = H;
     p.N = N;
     p.eta_over_n = (float)((double)eta / (double)N);
-    int smem = pool + extra;
-    // at most two CTAs per SM: their two 256-column TMEM allocations fill the 512 columns
-    smem = std::max(smem, dev->smem_per_sm / 3 + 1024);
+    // more than half an SM's shared memory: one CTA per SM, which owns all 512 TMEM columns
+    const int smem = std::max(p.slots * lin5::SLOT_BYTES + extra, dev->smem_per_sm / 2 + 1024);
     if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
 
-    CUtensorMap tk, tv, tq, tq128, to8, to32;
+    CUtensorMap tk, tv, tq, to;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!tmap_bf16_3d(&tk, k, 64, N, (int)U, p.TT, sw) || !tmap_bf16_3d(&tv, v, 64, N, (int)U, p.TT, sw) ||
-        !tmap_bf16_3d(&tq, q, 64, N, (int)U, p.TT, sw) || !tmap_bf16_3d(&tq128, q, 64, N, (int)U, lin5::MT, sw) ||
-        !tmap_bf16_3d(&to8, out, 64, N, (int)U, 8, sw) || !tmap_bf16_3d(&to32, out, 64, N, (int)U, 32, sw))
+        !tmap_bf16_3d(&tq, q, 64, N, (int)U, p.TT, sw) || !tmap_bf16_3d(&to, out, 64, N, (int)U, p.TT, sw))
         return TTT_ERR_CUDA;
     auto kern = lin5::linear_tc5_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess ||
@@ -251,14 +234,18 @@ int linear_tc5(const void* q, const void* k, const void* v, const float* w0, voi
     cfg.blockDim = dim3(lin5::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // the kernel may start while the previous grid on the stream finishes; it waits for that
+    // grid (griddepcontrol.wait) before its first global memory access
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, tq128, to8, to32, p) != cudaSuccess) return TTT_ERR_CUDA;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, to, p) != cudaSuccess) return TTT_ERR_CUDA;
     return launched(1);
 }
 
