@@ -33,8 +33,10 @@
 //      (deterministic, no atomics), forms W*^T rows = W0^T - (eta/N) grad^T in fp32 and sends
 //      them as bf16 hi + lo to every CTA of the cluster, again with st.async.
 //   4. Apply: Q tiles are loaded into the ring region, [O_hi | O_lo] = Q [W*_hi | W*_lo]
-//      (one N = 128 MMA chain per tile) into two TMEM buffers; the epilogue warps form two
-//      groups of four (one warp per lane quarter) that take alternate tiles: add the two
+//      (one N = 128 MMA chain per tile) into four TMEM buffers (all of TMEM: the Gram and
+//      W0^T G accumulators have been read by then); the Q tiles that fit are awaited while
+//      the exchange is in flight.  The epilogue warps form two groups of four (one warp per
+//      lane quarter) that take alternate tiles: add the two
 //      halves, write O as bf16 over the consumed Q tile, one TMA store per tile (rows >= N
 //      are clipped by the hardware).
 // Every wait is bounded (common.cuh).  Launched with programmatic stream serialization: the
@@ -60,8 +62,8 @@ constexpr int FIXED_BYTES = 4 * OP_BYTES + RECV_BYTES;  // W0 hi/lo, W* hi/lo, r
 constexpr int TMEM_COLS = 512;
 constexpr int COL_A = 0;                       // Gram accumulator [C^T ; G]
 constexpr int COL_D = 64;                      // W0^T [G_hi | G_lo] (rows 0-63), 128 columns
-constexpr int COL_O = 256;                     // two [O_hi | O_lo] buffers of 128 columns
-constexpr int OBUFS = 2;
+constexpr int COL_O = 0;                       // four [O_hi | O_lo] buffers of 128 columns (apply)
+constexpr int OBUFS = 4;
 constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
 constexpr uint32_t IDESC_WG = tc::idesc_bf16(128, 64, 0, 0);     // A K-major, B K-major
 constexpr uint32_t IDESC_WG2 = tc::idesc_bf16(128, 128, 0, 0);   // A K-major, B K-major, N = 128
@@ -265,6 +267,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
 
             // ---- apply: [O_hi | O_lo] = Q [W*_hi | W*_lo] per tile -----------------------------
+            const int q_first = n_t < NQ ? n_t : NQ;  // tiles whose Q is loaded up front
+            for (int t = 0; t < q_first; ++t) mbar_wait(&bars->qfull[t], 0, TTT_DEVERR_TIMEOUT_TMA);
             mbar_wait_cluster(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_PEER);   // the peers' W* rows
             mbar_wait(&bars->wlocal, 0, TTT_DEVERR_TIMEOUT_PEER);          // and this CTA's own
             fence_proxy_async_smem();  // W* rows were written by generic stores (local and st.async)
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int t = 0; t < n_t; ++t) {
                 const int b = t % OBUFS, qs = t % NQ;
                 if (t >= OBUFS) mbar_wait(&bars->tempty[b], (t / OBUFS - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-                mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                if (t >= q_first) mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 tc::fence_after();
                 const uint32_t qa = smem_u32(pool + qs * TILE_BYTES);
 #pragma unroll
