@@ -239,10 +239,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait(&bars->full[slot], (i / NS) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 tc::fence_after();
                 const uint32_t vb = smem_u32(pool + slot * SLOT_BYTES);
+                // A = [V | K]^T: MN-major, atoms V tile / K tile (LBO), 8-token groups (SBO); a
+                // k-step of 16 tokens moves both start addresses by 2 KB (start field += 128)
+                const uint64_t da = tc::smem_desc(vb, TILE_BYTES, 1024, 2);
+                const uint64_t db = tc::smem_desc(vb + TILE_BYTES, TILE_BYTES, 1024, 2);
                 for (int ks = 0; ks < TT / 16; ++ks)
-                    // A = [V | K]^T: MN-major, atoms V tile / K tile (LBO), 8-token groups (SBO)
-                    tc::mma_bf16(tmem + COL_A, tc::smem_desc(vb + ks * 2048, TILE_BYTES, 1024, 2),
-                                 tc::smem_desc(vb + TILE_BYTES + ks * 2048, TILE_BYTES, 1024, 2), IDESC_GRAM,
+                    tc::mma_bf16(tmem + COL_A, da + (uint64_t)(ks * 128), db + (uint64_t)(ks * 128), IDESC_GRAM,
                                  (i > 0 || ks > 0) ? 1 : 0);
                 tc::commit(&bars->empty[slot]);
             }
@@ -254,15 +256,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait(&bars->w0ready, 0, TTT_DEVERR_TIMEOUT_PEER);
                 mbar_wait(&bars->gready, 0, TTT_DEVERR_TIMEOUT_PEER);
                 tc::fence_after();
-                const uint32_t wa = smem_u32(w0op), ga = smem_u32(wsop);
+                // K-major operands: a k-step of 16 elements moves the start address by 32 B (+2)
+                const uint64_t dw = tc::smem_desc(smem_u32(w0op), 16, 1024, 2);
+                const uint64_t dwl = tc::smem_desc(smem_u32(w0op) + OP_BYTES, 16, 1024, 2);
+                const uint64_t dg = tc::smem_desc(smem_u32(wsop), 16, 1024, 2);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_D, tc::smem_desc(wa + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(ga + ks * 32, 16, 1024, 2), IDESC_WG2, ks > 0 ? 1 : 0);
+                    tc::mma_bf16(tmem + COL_D, dw + 2 * ks, dg + 2 * ks, IDESC_WG2, ks > 0 ? 1 : 0);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_D, tc::smem_desc(wa + OP_BYTES + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(ga + ks * 32, 16, 1024, 2), IDESC_WG, 1);
+                for (int ks = 0; ks < 4; ++ks) tc::mma_bf16(tmem + COL_D, dwl + 2 * ks, dg + 2 * ks, IDESC_WG, 1);
                 tc::commit(&bars->dfull);
             }
 
@@ -273,17 +275,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait(&bars->wlocal, 0, TTT_DEVERR_TIMEOUT_PEER);          // and this CTA's own
             fence_proxy_async_smem();  // W* rows were written by generic stores (local and st.async)
             tc::fence_after();
-            const uint32_t wsa = smem_u32(wsop);
+            const uint64_t dws = tc::smem_desc(smem_u32(wsop), 16, 1024, 2);
             for (int t = 0; t < n_t; ++t) {
                 const int b = t % OBUFS, qs = t % NQ;
                 if (t >= OBUFS) mbar_wait(&bars->tempty[b], (t / OBUFS - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
                 if (t >= q_first) mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 tc::fence_after();
-                const uint32_t qa = smem_u32(pool + qs * TILE_BYTES);
+                const uint64_t dq = tc::smem_desc(smem_u32(pool + qs * TILE_BYTES), 16, 1024, 2);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_O + b * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(wsa + ks * 32, 16, 1024, 2), IDESC_APPLY, ks > 0 ? 1 : 0);
+                    tc::mma_bf16(tmem + COL_O + b * 128, dq + 2 * ks, dws + 2 * ks, IDESC_APPLY, ks > 0 ? 1 : 0);
                 tc::commit(&bars->tfull[b]);
             }
         }
