@@ -48,18 +48,50 @@ __device__ __forceinline__ float tanh_fast(float x) {
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// gelu_tanh(u) and its derivative from the same t = tanh(sqrt(2/pi)(u + 0.044715 u^3))
-__device__ __forceinline__ float gelu_gp(float u, float* gp) {
-    const float s = 0.7978845608028654f, a = 0.044715f;
-    const float u2 = u * u;
-    const float t = tanh_fast(s * u * fmaf(a, u2, 1.f));
-    *gp = 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * s * fmaf(3.f * a, u2, 1.f);
-    return 0.5f * u * (1.f + t);
+// Packed fp32 pairs (one instruction for two lanes' worth of math: fma/mul/add.rn.f32x2).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
 }
-__device__ __forceinline__ float gelu_only(float u) {
-    const float s = 0.7978845608028654f, a = 0.044715f;
-    return 0.5f * u * (1.f + tanh_fast(s * u * fmaf(a, u * u, 1.f)));
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t tanh2(uint64_t x) { return pk2(tanh_fast(lo2(x)), tanh_fast(hi2(x))); }
+
+// gelu_tanh(u) = u/2 (1 + t), t = tanh(u s (1 + a u^2)), s = sqrt(2/pi), a = 0.044715, and its
+// derivative gelu'(u) = (1 + t)/2 + u/2 (1 - t^2) s (1 + 3 a u^2), for a pair of u:
+// ten packed operations and two hardware tanh per pair.
+__device__ __forceinline__ uint64_t gelu_gp2(uint64_t u, uint64_t* gp) {
+    const float s = 0.7978845608028654f, a = 0.044715f;
+    const uint64_t half = pk2(0.5f, 0.5f);
+    const uint64_t u2 = mul2(u, u);
+    const uint64_t t = tanh2(mul2(u, fma2(pk2(a * s, a * s), u2, pk2(s, s))));      // tanh(u s (1 + a u^2))
+    const uint64_t hu = mul2(u, half);
+    const uint64_t omt = fma2(t ^ 0x8000000080000000ull, t, pk2(1.f, 1.f));         // 1 - t^2
+    const uint64_t p = fma2(pk2(3.f * a * s, 3.f * a * s), u2, pk2(s, s));          // s (1 + 3 a u^2)
+    *gp = fma2(mul2(hu, omt), p, fma2(half, t, half));
+    return fma2(hu, t, hu);
+}
+__device__ __forceinline__ uint64_t gelu2(uint64_t u) {
+    const float s = 0.7978845608028654f, a = 0.044715f;
+    const uint64_t hu = mul2(u, pk2(0.5f, 0.5f));
+    const uint64_t t = tanh2(mul2(u, fma2(pk2(a * s, a * s), mul2(u, u), pk2(s, s))));
+    return fma2(hu, t, hu);
+}
+__device__ __forceinline__ uint32_t pack2_bf16(uint64_t v) { return pack_bf16(lo2(v), hi2(v)); }
 __device__ __forceinline__ void ld32(uint32_t taddr, float* v) {
     tc::ld16(taddr, v);
     tc::ld16(taddr + 16, v + 16);
@@ -71,41 +103,44 @@ __device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const f
 
 // ----------------------------------------------------------------------------- grad ----
 struct GradParams {
-    const float* w1;        // [H][64][256]
-    const float* w2;        // [H][256][64]
     const __nv_bfloat16* v; // [U][N][64]
-    float* part;            // [U][S][2][256][64]: gW1^T then gW2
+    float* part;            // [U][S][2][256][64]: gW1^T then gW2 (chunk-swizzled rows, see below)
     int H, N, T;            // T = tokens per CTA (multiple of 128)
 };
 
 struct GradBars {
-    uint64_t kfull[2], bfree[2], zfull, aready, pfull, rready, dafull, dzready, gdone;
+    uint64_t wfull, kfull[2], bfree[2], z0full, z1full, a0ready, a1ready, pfull, rready, da0full, da1full,
+        dz0ready, dz1ready, gdone;
     uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void load_weights(uint8_t* w1s, uint8_t* w2s, const float* w1, const float* w2, int tid,
-                                             int nthreads) {
-    // W1 [64][256] and W2 [256][64], fp32 -> bf16 swizzled; 8 consecutive elements per store
-    for (int e = tid; e < D * HID / 8; e += nthreads) {
-        const int k = e / (HID / 8), n = (e % (HID / 8)) * 8;
-        float v[8];
-        const float4 a = *reinterpret_cast<const float4*>(&w1[k * HID + n]);
-        const float4 b = *reinterpret_cast<const float4*>(&w1[k * HID + n + 4]);
-        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
-        store8_bf16(w1s, w1_off(k, n), v);
-    }
-    for (int e = tid; e < HID * D / 8; e += nthreads) {
-        const int h = e / (D / 8), d = (e % (D / 8)) * 8;
-        float v[8];
-        const float4 a = *reinterpret_cast<const float4*>(&w2[h * D + d]);
-        const float4 b = *reinterpret_cast<const float4*>(&w2[h * D + d + 4]);
-        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
-        store8_bf16(w2s, w2_off(h, d), v);
+// W1 [H][64][256] and W2 [H][256][64], fp32 -> bf16 (row-major), once per call, so that every
+// CTA can bring its head's weights into shared memory with five TMA loads.
+__global__ void __launch_bounds__(256) prep_kernel(const float* w1, const float* w2, __nv_bfloat16* w1h,
+                                                   __nv_bfloat16* w2h, int n8) {
+    for (int e = blockIdx.x * 256 + threadIdx.x; e < n8; e += gridDim.x * 256) {
+        const float* src = e < n8 / 2 ? w1 + (size_t)e * 8 : w2 + (size_t)(e - n8 / 2) * 8;
+        __nv_bfloat16* dst = e < n8 / 2 ? w1h + (size_t)e * 8 : w2h + (size_t)(e - n8 / 2) * 8;
+        const float4 a = *reinterpret_cast<const float4*>(src);
+        const float4 b = *reinterpret_cast<const float4*>(src + 4);
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
     }
 }
 
+// W1 (bf16 [idx][64][256]) as four 64 x 64 boxes -> the MN-major w1_off layout, W2 (bf16
+// [idx][256][64]) as one 256 x 64 box -> the w2_off layout; 128-byte swizzle, 64 KB on `bar`.
+__device__ __forceinline__ void tma_load_weights(uint8_t* w1s, uint8_t* w2s, const CUtensorMap* tw1,
+                                                 const CUtensorMap* tw2, int idx, uint64_t* bar) {
+    mbar_expect_tx(bar, 2 * WBYTES);
+#pragma unroll
+    for (int a = 0; a < HID / 64; ++a) tma_load_3d(w1s + a * 8192, tw1, a * 64, 0, idx, bar);
+    tma_load_3d(w2s, tw2, 0, 0, idx, bar);
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
-    grad_kernel(const __grid_constant__ CUtensorMap tm_k, const GradParams p) {
+    grad_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_w1,
+                const __grid_constant__ CUtensorMap tm_w2, const GradParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* w1s = smem;                 // 32 KB
@@ -123,22 +158,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int hd = u % p.H;
 
     if (threadIdx.x == 0) {
+        mbar_init(&bars->wfull, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->kfull[b], 1);
             mbar_init(&bars->bfree[b], 1);
         }
-        mbar_init(&bars->zfull, 1);
-        mbar_init(&bars->aready, EPI_WARPS);
+        mbar_init(&bars->z0full, 1);
+        mbar_init(&bars->z1full, 1);
+        mbar_init(&bars->a0ready, EPI_WARPS);
+        mbar_init(&bars->a1ready, EPI_WARPS);
         mbar_init(&bars->pfull, 1);
         mbar_init(&bars->rready, EPI_WARPS);
-        mbar_init(&bars->dafull, 1);
-        mbar_init(&bars->dzready, EPI_WARPS);
+        mbar_init(&bars->da0full, 1);
+        mbar_init(&bars->da1full, 1);
+        mbar_init(&bars->dz0ready, EPI_WARPS);
+        mbar_init(&bars->dz1ready, EPI_WARPS);
         mbar_init(&bars->gdone, 1);
         mbar_fence_init();
     }
-    load_weights(w1s, w2s, p.w1 + (size_t)hd * D * HID, p.w2 + (size_t)hd * HID * D, threadIdx.x, THREADS);
     if (warp == 1) tc::alloc(&bars->tmem_base, 512);
-    fence_proxy_async_smem();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
@@ -149,41 +187,58 @@ __global__ void __launch_bounds__(THREADS, 1)
         // tile i's K lives in buf[i & 1]; that buffer last held tile i-1's R, freed once the
         // MMAs reading R (gW2, dA) of tile i-1 completed (bfree)
         if (lane == 0) {
+            tma_load_weights(w1s, w2s, &tm_w1, &tm_w2, hd, &bars->wfull);
             for (int i = 0; i < ntiles; ++i) {
                 const int b = i & 1;
                 if (i >= 1) mbar_wait(&bars->bfree[b], ((i - 1) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 mbar_expect_tx(&bars->kfull[b], TILE);
                 tma_load_3d(buf + b * TILE, &tm_k, 0, t0 + i * MT, u, &bars->kfull[b]);
             }
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);  // no load in flight at exit
         }
     } else if (warp == 1) {
         // ================================ MMA issuer ===================================
+        // The 256 TMEM columns for Z / P / dA are two halves, T0 (hidden units 0-127, and P in
+        // its first 64 columns) and T1 (hidden units 128-255), so that the epilogue works on
+        // one half while the tensor cores fill the other.  Order per tile i:
+        //   P = A0 W2[0:128] (after a0ready), P += A1 W2[128:256] (after a1ready) -> pfull
+        //   gW2 += A^T R, dA0 = R W2[0:128]^T -> T0, dA1 = R W2[128:256]^T -> T1 (after rready)
+        //   gW1[0:128] += dZ0^T K (after dz0ready), then Z0 of tile i+1 -> T0,
+        //   gW1[128:256] += dZ1^T K (after dz1ready), then Z1 of tile i+1 -> T1.
+        // The tensor pipe runs MMAs in issue order, so a commit also covers every earlier MMA.
         if (lane == 0 && ntiles > 0) {
             const uint32_t w1a = smem_u32(w1s), w2a = smem_u32(w2s), aa = smem_u32(at), ga = smem_u32(gt);
-            const uint32_t IZ = tc::idesc_bf16(128, 256, 0, 1);   // K (K-major) x W1 (MN-major)
+            const uint32_t IZ = tc::idesc_bf16(128, 128, 0, 1);   // K (K-major) x W1 half (MN-major)
             const uint32_t IP = tc::idesc_bf16(128, 64, 0, 1);    // A (K-major) x W2 (MN-major)
             const uint32_t IG = tc::idesc_bf16(128, 64, 1, 1);    // A^T/dZ^T (MN-major) x R/K (MN-major)
-            const uint32_t ID = tc::idesc_bf16(128, 256, 0, 0);   // R (K-major) x W2^T (K-major)
+            const uint32_t ID = tc::idesc_bf16(128, 128, 0, 0);   // R (K-major) x W2^T half (K-major)
+            auto issue_z = [&](int i, int half) {  // Z half of tile i: K W1[:, 128 half ..]
+                const uint32_t kb = smem_u32(buf + (i & 1) * TILE);
+                tc::fence_after();
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(kb + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(w1a + half * 2 * 8192 + ks * 2048, 8192, 1024, 2), IZ, ks > 0);
+                tc::commit(half ? &bars->z1full : &bars->z0full);
+            };
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+            mbar_wait(&bars->kfull[0], 0, TTT_DEVERR_TIMEOUT_TMA);
+            issue_z(0, 0);
+            issue_z(0, 1);
             for (int i = 0; i < ntiles; ++i) {
                 const int b = i & 1;
                 const uint32_t kb = smem_u32(buf + b * TILE), rb = smem_u32(buf + (b ^ 1) * TILE);
                 const uint32_t ph = i & 1;
-                // Z = K W1  (T region, 256 columns)
-                mbar_wait(&bars->kfull[b], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
-                if (i > 0) mbar_wait(&bars->dzready, (i - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);  // T free
-                tc::fence_after();
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_T, tc::smem_desc(kb + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(w1a + ks * 2048, 8192, 1024, 2), IZ, ks > 0);
-                tc::commit(&bars->zfull);
-                // P = A W2  (T columns 0..63)
-                mbar_wait(&bars->aready, ph, TTT_DEVERR_TIMEOUT_PEER);
-                tc::fence_after();
-                for (int ks = 0; ks < 16; ++ks)
-                    tc::mma_bf16(tmem + COL_T, tc::smem_desc(aa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
-                                 tc::smem_desc(w2a + ks * 2048, 8192, 1024, 2), IP, ks > 0);
+                // P = A W2 in two K halves (T0 columns 0..63)
+                for (int half = 0; half < 2; ++half) {
+                    mbar_wait(half ? &bars->a1ready : &bars->a0ready, ph, TTT_DEVERR_TIMEOUT_PEER);
+                    tc::fence_after();
+                    for (int ks = half * 8; ks < half * 8 + 8; ++ks)
+                        tc::mma_bf16(tmem + COL_T,
+                                     tc::smem_desc(aa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
+                                     tc::smem_desc(w2a + ks * 2048, 8192, 1024, 2), IP, ks > 0);
+                }
                 tc::commit(&bars->pfull);
-                // gW2 += A^T R (two 128-row halves of h) and dA = R W2^T (T region)
+                // gW2 += A^T R (two 128-row halves of h); dA0 -> T0, dA1 -> T1
                 mbar_wait(&bars->rready, ph, TTT_DEVERR_TIMEOUT_PEER);
                 tc::fence_after();
                 for (int hh = 0; hh < 2; ++hh)
@@ -191,19 +246,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tc::mma_bf16(tmem + COL_G2 + hh * 64,
                                      tc::smem_desc(aa + hh * 2 * 16384 + ks * 2048, 16384, 1024, 2),
                                      tc::smem_desc(rb + ks * 2048, 8192, 1024, 2), IG, (i > 0 || ks > 0));
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_T, tc::smem_desc(rb + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(w2a + ks * 32, 16, 1024, 2), ID, ks > 0);
-                tc::commit(&bars->dafull);
+                for (int half = 0; half < 2; ++half) {
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(rb + ks * 32, 16, 1024, 2),
+                                     tc::smem_desc(w2a + half * 16384 + ks * 32, 16, 1024, 2), ID, ks > 0);
+                    tc::commit(half ? &bars->da1full : &bars->da0full);
+                }
                 tc::commit(&bars->bfree[b ^ 1]);  // R buffer free once these MMAs completed
-                // gW1^T += dZ^T K
-                mbar_wait(&bars->dzready, ph, TTT_DEVERR_TIMEOUT_PEER);
-                tc::fence_after();
-                for (int hh = 0; hh < 2; ++hh)
+                // gW1^T += dZ^T K per half of h; the freed T half takes the next tile's Z half
+                for (int hh = 0; hh < 2; ++hh) {
+                    mbar_wait(hh ? &bars->dz1ready : &bars->dz0ready, ph, TTT_DEVERR_TIMEOUT_PEER);
+                    tc::fence_after();
                     for (int ks = 0; ks < 8; ++ks)
                         tc::mma_bf16(tmem + COL_G1 + hh * 64,
                                      tc::smem_desc(ga + hh * 2 * 16384 + ks * 2048, 16384, 1024, 2),
                                      tc::smem_desc(kb + ks * 2048, 8192, 1024, 2), IG, (i > 0 || ks > 0));
+                    if (i + 1 < ntiles) {
+                        if (hh == 0) mbar_wait(&bars->kfull[b ^ 1], ((i + 1) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                        issue_z(i + 1, hh);
+                    }
+                }
             }
             tc::commit(&bars->gdone);
         }
@@ -225,26 +287,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int c = 0; c < 4; ++c)
                 vv[c] = tok < p.N ? *reinterpret_cast<const uint4*>(vu + (size_t)tok * D + ch * 32 + c * 8)
                                   : make_uint4(0, 0, 0, 0);
-            // ---- Z -> A = gelu(Z), gelu'(Z) -------------------------------------------------
-            mbar_wait(&bars->zfull, ph, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
-            for (int c0 = ch * 128; c0 < ch * 128 + 128; c0 += 32) {
-                float z[32];
-                ld32(lane_base + COL_T + c0, z);
-                tc::wait_ld();
-                float a[32], g[32];
+            // ---- Z half -> A = gelu(Z), gelu'(Z), hidden units [128 half, 128 half + 128) -----
+            // this warp: 64 of those columns (ch), lanes = its 32 token rows
+            for (int half = 0; half < 2; ++half) {
+                mbar_wait(half ? &bars->z1full : &bars->z0full, ph, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
+                {
+                    const int c0 = half * 128 + ch * 64;  // 64 columns, one TMEM round trip
+                    float z[64];
+                    ld32(lane_base + COL_T + c0, z);
+                    ld32(lane_base + COL_T + c0 + 32, z + 32);
+                    tc::wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) a[j] = gelu_gp(z[j], &g[j]);
+                    for (int j = 0; j < 64; j += 8) {
+                        uint32_t a[4], g[4];
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    store8_bf16(at, big_off(r, c0 + j), &a[j]);
-                    store8_bf16(gt, big_off(r, c0 + j), &g[j]);
+                        for (int e = 0; e < 4; ++e) {
+                            uint64_t gp;
+                            a[e] = pack2_bf16(gelu_gp2(pk2(z[j + 2 * e], z[j + 2 * e + 1]), &gp));
+                            g[e] = pack2_bf16(gp);
+                        }
+                        *reinterpret_cast<uint4*>(at + big_off(r, c0 + j)) = make_uint4(a[0], a[1], a[2], a[3]);
+                        *reinterpret_cast<uint4*>(gt + big_off(r, c0 + j)) = make_uint4(g[0], g[1], g[2], g[3]);
+                    }
                 }
+                fence_proxy_async_smem();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(half ? &bars->a1ready : &bars->a0ready);
             }
-            fence_proxy_async_smem();
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->aready);
             // ---- P -> R = P - V ---------------------------------------------------------------
             mbar_wait(&bars->pfull, ph, TTT_DEVERR_TIMEOUT_PEER);
             tc::fence_after();
@@ -271,31 +342,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->rready);
-            // ---- dA -> dZ = dA * gelu'(Z), in place over gelu'(Z) --------------------------------
-            mbar_wait(&bars->dafull, ph, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
-            for (int c0 = ch * 128; c0 < ch * 128 + 128; c0 += 32) {
-                float da[32];
-                ld32(lane_base + COL_T + c0, da);
-                tc::wait_ld();
+            // ---- dA half -> dZ = dA * gelu'(Z), in place over gelu'(Z) ---------------------------
+            for (int half = 0; half < 2; ++half) {
+                mbar_wait(half ? &bars->da1full : &bars->da0full, ph, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
+                {
+                    const int c0 = half * 128 + ch * 64;  // 64 columns, one TMEM round trip
+                    float da[64];
+                    ld32(lane_base + COL_T + c0, da);
+                    ld32(lane_base + COL_T + c0 + 32, da + 32);
+                    tc::wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    const uint32_t off = big_off(r, c0 + j);
-                    const uint4 gq = *reinterpret_cast<const uint4*>(gt + off);
-                    const uint32_t w[4] = {gq.x, gq.y, gq.z, gq.w};
-                    float dz[8];
+                    for (int j = 0; j < 64; j += 8) {
+                        const uint32_t off = big_off(r, c0 + j);
+                        const uint4 gq = *reinterpret_cast<const uint4*>(gt + off);
+                        const uint32_t w[4] = {gq.x, gq.y, gq.z, gq.w};
+                        float dz[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        dz[2 * e] = da[j + 2 * e] * __uint_as_float(w[e] << 16);
-                        dz[2 * e + 1] = da[j + 2 * e + 1] * __uint_as_float(w[e] & 0xffff0000u);
+                        for (int e = 0; e < 4; ++e) {
+                            dz[2 * e] = da[j + 2 * e] * __uint_as_float(w[e] << 16);
+                            dz[2 * e + 1] = da[j + 2 * e + 1] * __uint_as_float(w[e] & 0xffff0000u);
+                        }
+                        store8_bf16(gt, off, dz);
                     }
-                    store8_bf16(gt, off, dz);
                 }
+                fence_proxy_async_smem();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(half ? &bars->dz1ready : &bars->dz0ready);
             }
-            fence_proxy_async_smem();
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dzready);
         }
         // ---- partial gradients: TMEM -> workspace --------------------------------------------
         float* part = p.part + ((size_t)u * S + split) * 2 * HID * D;
@@ -303,24 +378,40 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait(&bars->gdone, 0, TTT_DEVERR_TIMEOUT_PEER);
             tc::fence_after();
         }
-        // TMEM lane = h row within a 128-row half; this warp: half ch, rows q4*32 + lane
+        // TMEM lane = h row within a 128-row half; this warp: half ch, rows q4*32 + lane.
+        // Both gradients are staged in the (now idle) A and gelu' buffers, 64 KB each, and
+        // leave with one bulk copy apiece.  Row h keeps its 16 float4 chunks at positions
+        // c ^ (h & 7) (the workspace layout; the update kernel reads it back the same way), so
+        // that the 32 rows a warp writes spread over all banks.
         const int hrow = ch * 128 + r;
-        for (int which = 0; which < 2; ++which) {  // 0: gW1^T, 1: gW2
+        for (int which = 0; which < 2; ++which) {  // 0: gW1^T -> at, 1: gW2 -> gt
             const uint32_t col = (which == 0 ? COL_G1 : COL_G2) + ch * 64;
-            float* dst = part + (size_t)which * HID * D + (size_t)hrow * D;
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                float g[32];
-                if (ntiles > 0) {
-                    ld32(lane_base + col + c0, g);
-                    tc::wait_ld();
-                } else {
+            float* srow = reinterpret_cast<float*>(which == 0 ? at : gt) + (size_t)hrow * D;
+            float g[64];
+            if (ntiles > 0) {
+                ld32(lane_base + col, g);
+                ld32(lane_base + col + 32, g + 32);
+                tc::wait_ld();
+            } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) g[j] = 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(g[j], g[j + 1], g[j + 2], g[j + 3]);
+                for (int j = 0; j < 64; ++j) g[j] = 0.f;
             }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<float4*>(srow + 4 * (c ^ (hrow & 7))) =
+                    make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
+        }
+        fence_proxy_async_smem();  // read next by the bulk copies
+        asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
+        if (warp == 2 && lane == 0) {
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(part),
+                         "r"(smem_u32(at)), "r"(HID * D * 4)
+                         : "memory");
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(part + HID * D),
+                         "r"(smem_u32(gt)), "r"(HID * D * 4)
+                         : "memory");
+            tma_store_commit();
+            tma_store_wait_all();
         }
     }
     tc::fence_before();
@@ -346,10 +437,12 @@ __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
     const float* part = p.part + (size_t)u * p.S * 2 * HID * D;
     for (int e = threadIdx.x + blockIdx.y * 256; e < HID * D; e += 256 * gridDim.y) {
         const int hr = e / D, dc = e % D;  // element (h, d) of gW1^T and gW2
+        // position of (h, d) in a partial: float4 chunk (d / 4) ^ (h & 7) of row h
+        const int pe = hr * D + ((((dc >> 2) ^ (hr & 7))) << 2) + (dc & 3);
         float g1 = 0.f, g2 = 0.f;
         for (int s = 0; s < p.S; ++s) {   // split order
-            g1 += part[(size_t)s * 2 * HID * D + e];
-            g2 += part[(size_t)s * 2 * HID * D + HID * D + e];
+            g1 += part[(size_t)s * 2 * HID * D + pe];
+            g2 += part[(size_t)s * 2 * HID * D + HID * D + pe];
         }
         const float w1 = p.w1[(size_t)hd * D * HID + dc * HID + hr] - p.eta_over_n * g1;  // W1*[d][h]
         const float w2 = p.w2[(size_t)hd * HID * D + e] - p.eta_over_n * g2;              // W2*[h][d]
@@ -362,18 +455,18 @@ __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
 
 // ----------------------------------------------------------------------------- apply ---
 struct ApplyParams {
-    const __nv_bfloat16* w1b;  // [U][64][256]
-    const __nv_bfloat16* w2b;  // [U][256][64]
     int N, T;
 };
 
 struct ApplyBars {
-    uint64_t qfull[2], qfree[2], zfull, aready, ofull, oread;
+    uint64_t wfull, qfull[2], qfree[2], z0full, z1full, a0ready, a1ready, ofull[2], oread[2];
     uint32_t tmem_base;
 };
+constexpr uint32_t COL_O = 256;  // apply: two 64-column O buffers after the two Z halves
 
 __global__ void __launch_bounds__(THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                 const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
                  const ApplyParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -390,30 +483,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ntiles = (n_valid + MT - 1) / MT;
 
     if (threadIdx.x == 0) {
+        mbar_init(&bars->wfull, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->qfull[b], 1);
             mbar_init(&bars->qfree[b], EPI_WARPS);
         }
-        mbar_init(&bars->zfull, 1);
-        mbar_init(&bars->aready, EPI_WARPS);
-        mbar_init(&bars->ofull, 1);
-        mbar_init(&bars->oread, EPI_WARPS);
+        mbar_init(&bars->z0full, 1);
+        mbar_init(&bars->z1full, 1);
+        mbar_init(&bars->a0ready, EPI_WARPS);
+        mbar_init(&bars->a1ready, EPI_WARPS);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->ofull[b], 1);
+            mbar_init(&bars->oread[b], EPI_WARPS);
+        }
         mbar_fence_init();
     }
-    {   // W1*, W2* (bf16) -> swizzled shared memory
-        const __nv_bfloat16* w1 = p.w1b + (size_t)u * D * HID;
-        const __nv_bfloat16* w2 = p.w2b + (size_t)u * HID * D;
-        for (int e = threadIdx.x; e < D * HID / 8; e += THREADS) {
-            const int k = e / (HID / 8), n = (e % (HID / 8)) * 8;
-            *reinterpret_cast<uint4*>(w1s + w1_off(k, n)) = *reinterpret_cast<const uint4*>(w1 + k * HID + n);
-        }
-        for (int e = threadIdx.x; e < HID * D / 8; e += THREADS) {
-            const int h = e / (D / 8), d = (e % (D / 8)) * 8;
-            *reinterpret_cast<uint4*>(w2s + w2_off(h, d)) = *reinterpret_cast<const uint4*>(w2 + h * D + d);
-        }
-    }
     if (warp == 1) tc::alloc(&bars->tmem_base, 512);
-    fence_proxy_async_smem();
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
@@ -421,34 +506,50 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            tma_load_weights(w1s, w2s, &tm_w1, &tm_w2, u, &bars->wfull);  // this unit's W1*, W2*
             for (int i = 0; i < ntiles; ++i) {
                 const int b = i & 1;
                 if (i >= 2) mbar_wait(&bars->qfree[b], ((i - 2) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 mbar_expect_tx(&bars->qfull[b], TILE);
                 tma_load_3d(qb + b * TILE, &tm_q, 0, t0 + i * MT, u, &bars->qfull[b]);
             }
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);  // no load in flight at exit
         }
     } else if (warp == 1) {
+        // Z in two hidden halves (T0, T1) and O in two buffers: Z0 of tile i+1 is issued once
+        // the epilogue has read Z0 of tile i, while it still works on Z1 and on O of tile i.
         if (lane == 0 && ntiles > 0) {
             const uint32_t w1a = smem_u32(w1s), w2a = smem_u32(w2s), aa = smem_u32(at);
-            const uint32_t IZ = tc::idesc_bf16(128, 256, 0, 1);
+            const uint32_t IZ = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t IO = tc::idesc_bf16(128, 64, 0, 1);
-            for (int i = 0; i < ntiles; ++i) {
-                const int b = i & 1;
-                mbar_wait(&bars->qfull[b], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
-                if (i > 0) mbar_wait(&bars->oread, (i - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);  // TMEM free
+            auto issue_z = [&](int i, int half) {
+                const uint32_t qa = smem_u32(qb + (i & 1) * TILE);
                 tc::fence_after();
-                const uint32_t qa = smem_u32(qb + b * TILE);
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_T, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
-                                 tc::smem_desc(w1a + ks * 2048, 8192, 1024, 2), IZ, ks > 0);
-                tc::commit(&bars->zfull);
-                mbar_wait(&bars->aready, i & 1, TTT_DEVERR_TIMEOUT_PEER);
-                tc::fence_after();
-                for (int ks = 0; ks < 16; ++ks)
-                    tc::mma_bf16(tmem + COL_G2, tc::smem_desc(aa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
-                                 tc::smem_desc(w2a + ks * 2048, 8192, 1024, 2), IO, ks > 0);
-                tc::commit(&bars->ofull);
+                    tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(w1a + half * 2 * 8192 + ks * 2048, 8192, 1024, 2), IZ, ks > 0);
+                tc::commit(half ? &bars->z1full : &bars->z0full);
+            };
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+            mbar_wait(&bars->qfull[0], 0, TTT_DEVERR_TIMEOUT_TMA);
+            issue_z(0, 0);
+            issue_z(0, 1);
+            for (int i = 0; i < ntiles; ++i) {
+                const int ob = i & 1;
+                if (i >= 2) mbar_wait(&bars->oread[ob], ((i - 2) >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                for (int half = 0; half < 2; ++half) {
+                    mbar_wait(half ? &bars->a1ready : &bars->a0ready, i & 1, TTT_DEVERR_TIMEOUT_PEER);
+                    tc::fence_after();
+                    for (int ks = half * 8; ks < half * 8 + 8; ++ks)
+                        tc::mma_bf16(tmem + COL_O + ob * 64,
+                                     tc::smem_desc(aa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
+                                     tc::smem_desc(w2a + ks * 2048, 8192, 1024, 2), IO, ks > 0);
+                    if (half) tc::commit(&bars->ofull[ob]);
+                    if (i + 1 < ntiles) {
+                        if (half == 0) mbar_wait(&bars->qfull[(i + 1) & 1], ((i + 1) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                        issue_z(i + 1, half);
+                    }
+                }
             }
         }
     } else {
@@ -456,29 +557,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r = q4 * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         for (int i = 0; i < ntiles; ++i) {
-            const int b = i & 1;
+            const int b = i & 1, ob = i & 1;
             uint8_t* tile = qb + b * TILE;
-            mbar_wait(&bars->zfull, i & 1, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
-            for (int c0 = ch * 128; c0 < ch * 128 + 128; c0 += 32) {
-                float z[32];
+            for (int half = 0; half < 2; ++half) {  // A = gelu(Z), 64 columns per warp and half
+                mbar_wait(half ? &bars->z1full : &bars->z0full, i & 1, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
+                const int c0 = half * 128 + ch * 64;
+                float z[64];
                 ld32(lane_base + COL_T + c0, z);
+                ld32(lane_base + COL_T + c0 + 32, z + 32);
                 tc::wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) z[j] = gelu_only(z[j]);
+                for (int j = 0; j < 64; j += 8) {
+                    uint32_t a[4];
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) store8_bf16(at, big_off(r, c0 + j), &z[j]);
+                    for (int e = 0; e < 4; ++e) a[e] = pack2_bf16(gelu2(pk2(z[j + 2 * e], z[j + 2 * e + 1])));
+                    *reinterpret_cast<uint4*>(at + big_off(r, c0 + j)) = make_uint4(a[0], a[1], a[2], a[3]);
+                }
+                fence_proxy_async_smem();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(half ? &bars->a1ready : &bars->a0ready);
             }
-            fence_proxy_async_smem();
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->aready);
-            // O = A W2* -> bf16 over the Q tile (its MMA finished before zfull) -> TMA store
-            mbar_wait(&bars->ofull, i & 1, TTT_DEVERR_TIMEOUT_PEER);
+            // O = A W2* -> bf16 over the Q tile (the Z MMAs that read it have completed) -> TMA
+            mbar_wait(&bars->ofull[ob], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             tc::fence_after();
             {
                 float o[32];
-                ld32(lane_base + COL_G2 + ch * 32, o);
+                ld32(lane_base + COL_O + ob * 64 + ch * 32, o);
                 tc::wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) store8_bf16(tile, swz<3>(r * ROWB + (ch * 32 + j) * 2), &o[j]);
@@ -486,14 +592,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::fence_before();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars->oread);
-                // rows q4*32 .. +31 of this tile, columns of this half are written by this warp;
-                // the other half's warp writes the other 32 columns: one store per row-quarter
-                // is issued by the ch == 0 warp after both halves have arrived (oread phase)
-            }
-            // wait until both column halves of this row quarter are in shared memory
-            mbar_wait(&bars->oread, i & 1, TTT_DEVERR_TIMEOUT_PEER);
+            if (lane == 0) mbar_arrive(&bars->oread[ob]);
+            // both column halves of every row quarter are in shared memory once oread completes
+            mbar_wait(&bars->oread[ob], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             if (ch == 0 && lane == 0) {
                 const int row0 = i * MT + q4 * 32;
                 if (row0 < n_valid) {

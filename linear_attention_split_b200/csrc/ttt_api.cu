@@ -99,6 +99,21 @@ bool tmap_bf16_3d(CUtensorMap* m, const void* base, int d, int N, int U, int box
 }
 
 // ------------------------------------------------------------------ TTT-Linear --------
+// bf16 tensor [dim2][dim1][dim0] (dim0 fastest) viewed as 3-D, box {box0, box1, 1}
+bool tmap_bf16_box(CUtensorMap* m, const void* base, int dim0, int dim1, int dim2, int box0, int box1,
+                   CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
+    cuuint64_t strides[2] = {(cuuint64_t)dim0 * 2, (cuuint64_t)dim1 * dim0 * 2};
+    cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool linear_uses_tc(int d, int dtype) { return dtype == TTT_BF16 && (d == 32 || d == 64); }
 
 template <typename T>
@@ -409,7 +424,8 @@ size_t mlp_tc_ws(int B, int H, int N) {
     const int sms = current_device(&dev) == TTT_OK ? dev->sms : 148;
     const long long U = (long long)B * H;
     const int S = mlp_splits(U, N, sms);
-    return align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4) + 2 * align256((size_t)U * mlp::D * mlp::HID * 2);
+    return align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4) + 2 * align256((size_t)U * mlp::D * mlp::HID * 2) +
+           2 * align256((size_t)H * mlp::D * mlp::HID * 2);
 }
 
 int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
@@ -425,11 +441,19 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(w);
     w += align256((size_t)U * mlp::D * mlp::HID * 2);
     __nv_bfloat16* w2b = reinterpret_cast<__nv_bfloat16*>(w);
+    w += align256((size_t)U * mlp::D * mlp::HID * 2);
+    __nv_bfloat16* w1h = reinterpret_cast<__nv_bfloat16*>(w);   // W1, W2 of every head in bf16
+    w += align256((size_t)H * mlp::D * mlp::HID * 2);
+    __nv_bfloat16* w2h = reinterpret_cast<__nv_bfloat16*>(w);
 
-    CUtensorMap tk, tq, to;
-    if (!tmap_bf16_3d(&tk, k, 64, N, U, mlp::MT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tmap_bf16_3d(&tq, q, 64, N, U, mlp::MT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tmap_bf16_3d(&to, out, 64, N, U, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    CUtensorMap tk, tq, to, tw1h, tw2h, tw1s, tw2s;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!tmap_bf16_3d(&tk, k, 64, N, U, mlp::MT, sw) || !tmap_bf16_3d(&tq, q, 64, N, U, mlp::MT, sw) ||
+        !tmap_bf16_3d(&to, out, 64, N, U, 32, sw) ||
+        !tmap_bf16_box(&tw1h, w1h, mlp::HID, mlp::D, H, 64, 64, sw) ||
+        !tmap_bf16_box(&tw2h, w2h, mlp::D, mlp::HID, H, 64, mlp::HID, sw) ||
+        !tmap_bf16_box(&tw1s, w1b, mlp::HID, mlp::D, U, 64, 64, sw) ||
+        !tmap_bf16_box(&tw2s, w2b, mlp::D, mlp::HID, U, 64, mlp::HID, sw))
         return TTT_ERR_CUDA;
     const int smem_g = 2 * mlp::WBYTES + 2 * mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::GradBars) + 1024;
     const int smem_a = 2 * mlp::WBYTES + mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
@@ -437,15 +461,15 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     if (cudaFuncSetAttribute(mlp::grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_g) != cudaSuccess ||
         cudaFuncSetAttribute(mlp::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
         return TTT_ERR_CUDA;
+    const int n8 = H * mlp::D * mlp::HID * 2 / 8;  // 8-element groups of W1 and W2
+    mlp::prep_kernel<<<(n8 + 255) / 256, 256, 0, st>>>(w1, w2, w1h, w2h, n8);
     mlp::GradParams gp;
-    gp.w1 = w1;
-    gp.w2 = w2;
     gp.v = static_cast<const __nv_bfloat16*>(v);
     gp.part = part;
     gp.H = H;
     gp.N = N;
     gp.T = T;
-    mlp::grad_kernel<<<dim3(S, U), mlp::THREADS, smem_g, st>>>(tk, gp);
+    mlp::grad_kernel<<<dim3(S, U), mlp::THREADS, smem_g, st>>>(tk, tw1h, tw2h, gp);
     mlp::UpdateParams up;
     up.w1 = w1;
     up.w2 = w2;
@@ -459,12 +483,10 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     up.eta_over_n = (float)((double)eta / (double)N);
     mlp::update_kernel<<<dim3(U, 8), 256, 0, st>>>(up);
     mlp::ApplyParams ap;
-    ap.w1b = w1b;
-    ap.w2b = w2b;
     ap.N = N;
     ap.T = T;
-    mlp::apply_kernel<<<dim3(S, U), mlp::THREADS, smem_a, st>>>(tq, to, ap);
-    return launched(3);
+    mlp::apply_kernel<<<dim3(S, U), mlp::THREADS, smem_a, st>>>(tq, to, tw1s, tw2s, ap);
+    return launched(4);
 }
 
 // ------------------------------------------------------------------ chunked scan ------
