@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // its first 64 columns) and T1 (hidden units 128-255), so that the epilogue works on
         // one half while the tensor cores fill the other.  Order per tile i:
         //   P = A0 W2[0:128] (after a0ready), P += A1 W2[128:256] (after a1ready) -> pfull
-        //   gW2 += A^T R, dA0 = R W2[0:128]^T -> T0, dA1 = R W2[128:256]^T -> T1 (after rready)
+        //   dA0 = R W2[0:128]^T -> T0, dA1 = R W2[128:256]^T -> T1, then gW2 += A^T R (after rready)
         //   gW1[0:128] += dZ0^T K (after dz0ready), then Z0 of tile i+1 -> T0,
         //   gW1[128:256] += dZ1^T K (after dz1ready), then Z1 of tile i+1 -> T1.
         // The tensor pipe runs MMAs in issue order, so a commit also covers every earlier MMA.
@@ -241,17 +241,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // gW2 += A^T R (two 128-row halves of h); dA0 -> T0, dA1 -> T1
                 mbar_wait(&bars->rready, ph, TTT_DEVERR_TIMEOUT_PEER);
                 tc::fence_after();
-                for (int hh = 0; hh < 2; ++hh)
-                    for (int ks = 0; ks < 8; ++ks)
-                        tc::mma_bf16(tmem + COL_G2 + hh * 64,
-                                     tc::smem_desc(aa + hh * 2 * 16384 + ks * 2048, 16384, 1024, 2),
-                                     tc::smem_desc(rb + ks * 2048, 8192, 1024, 2), IG, (i > 0 || ks > 0));
-                for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < 2; ++half) {  // dA first: the epilogue waits for it
                     for (int ks = 0; ks < 4; ++ks)
                         tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(rb + ks * 32, 16, 1024, 2),
                                      tc::smem_desc(w2a + half * 16384 + ks * 32, 16, 1024, 2), ID, ks > 0);
                     tc::commit(half ? &bars->da1full : &bars->da0full);
                 }
+                for (int hh = 0; hh < 2; ++hh)
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc::mma_bf16(tmem + COL_G2 + hh * 64,
+                                     tc::smem_desc(aa + hh * 2 * 16384 + ks * 2048, 16384, 1024, 2),
+                                     tc::smem_desc(rb + ks * 2048, 8192, 1024, 2), IG, (i > 0 || ks > 0));
                 tc::commit(&bars->bfree[b ^ 1]);  // R buffer free once these MMAs completed
                 // gW1^T += dZ^T K per half of h; the freed T half takes the next tile's Z half
                 for (int hh = 0; hh < 2; ++hh) {
