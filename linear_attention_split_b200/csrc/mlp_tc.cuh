@@ -432,24 +432,34 @@ struct UpdateParams {
     float eta_over_n;
 };
 
+// Block (u, c): rows h in [64 c, 64 c + 64) of gW1^T and gW2.  The S partials are added in
+// split order (deterministic).  W2*[h][d] is written row by row; W1*[d][h] is the transpose of
+// the gW1^T block, so that block goes through shared memory and leaves row by row as well.
 __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
-    const int u = blockIdx.x, hd = u % p.H;
+    __shared__ float tile[64][65];  // W1*^T block: [h - h0][d]
+    const int u = blockIdx.x, hd = u % p.H, h0 = blockIdx.y * 64;
     const float* part = p.part + (size_t)u * p.S * 2 * HID * D;
-    for (int e = threadIdx.x + blockIdx.y * 256; e < HID * D; e += 256 * gridDim.y) {
-        const int hr = e / D, dc = e % D;  // element (h, d) of gW1^T and gW2
-        // position of (h, d) in a partial: float4 chunk (d / 4) ^ (h & 7) of row h
-        const int pe = hr * D + ((((dc >> 2) ^ (hr & 7))) << 2) + (dc & 3);
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 columns x 4 rows per pass
+    for (int rr = ty; rr < 64; rr += 4) {
+        const int h = h0 + rr;
+        // element (h, d = tx): float4 chunk (tx / 4) ^ (h & 7) of row h in a partial
+        const int pe = h * D + ((((tx >> 2) ^ (h & 7))) << 2) + (tx & 3);
         float g1 = 0.f, g2 = 0.f;
-        for (int s = 0; s < p.S; ++s) {   // split order
-            g1 += part[(size_t)s * 2 * HID * D + pe];
-            g2 += part[(size_t)s * 2 * HID * D + HID * D + pe];
+        for (int sp = 0; sp < p.S; ++sp) {  // split order
+            g1 += part[(size_t)sp * 2 * HID * D + pe];
+            g2 += part[(size_t)sp * 2 * HID * D + HID * D + pe];
         }
-        const float w1 = p.w1[(size_t)hd * D * HID + dc * HID + hr] - p.eta_over_n * g1;  // W1*[d][h]
-        const float w2 = p.w2[(size_t)hd * HID * D + e] - p.eta_over_n * g2;              // W2*[h][d]
-        if (p.w1_star) p.w1_star[(size_t)u * D * HID + dc * HID + hr] = w1;
-        if (p.w2_star) p.w2_star[(size_t)u * HID * D + e] = w2;
-        p.w1b[(size_t)u * D * HID + dc * HID + hr] = __float2bfloat16_rn(w1);
-        p.w2b[(size_t)u * HID * D + e] = __float2bfloat16_rn(w2);
+        const float w2 = p.w2[(size_t)hd * HID * D + h * D + tx] - p.eta_over_n * g2;  // W2*[h][d]
+        if (p.w2_star) p.w2_star[(size_t)u * HID * D + h * D + tx] = w2;
+        p.w2b[(size_t)u * HID * D + h * D + tx] = __float2bfloat16_rn(w2);
+        tile[rr][tx] = g1;  // gW1^T[h][d]
+    }
+    __syncthreads();
+    for (int dd = ty; dd < 64; dd += 4) {  // W1*[d][h0 + tx]
+        const size_t idx = (size_t)dd * HID + h0 + tx;
+        const float w1 = p.w1[(size_t)hd * D * HID + idx] - p.eta_over_n * tile[tx][dd];
+        if (p.w1_star) p.w1_star[(size_t)u * D * HID + idx] = w1;
+        p.w1b[(size_t)u * D * HID + idx] = __float2bfloat16_rn(w1);
     }
 }
 

@@ -481,7 +481,7 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     up.H = H;
     up.S = S;
     up.eta_over_n = (float)((double)eta / (double)N);
-    mlp::update_kernel<<<dim3(U, 8), 256, 0, st>>>(up);
+    mlp::update_kernel<<<dim3(U, mlp::HID / 64), 256, 0, st>>>(up);
     mlp::ApplyParams ap;
     ap.N = N;
     ap.T = T;
