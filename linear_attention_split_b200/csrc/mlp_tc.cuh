@@ -469,10 +469,11 @@ struct ApplyParams {
 };
 
 struct ApplyBars {
-    uint64_t wfull, qfull[2], qfree[2], z0full, z1full, a0ready, a1ready, ofull[2], oread[2];
+    uint64_t wfull, qfull[4], qfree[4], z0full, z1full, a0ready, a1ready, ofull[2], oread[2];
     uint32_t tmem_base;
 };
 constexpr uint32_t COL_O = 256;  // apply: two 64-column O buffers after the two Z halves
+constexpr int NQB = 4;           // apply: Q tile buffers (O of a tile is staged over its Q tile)
 
 __global__ void __launch_bounds__(THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
@@ -483,8 +484,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* w1s = smem;
     uint8_t* w2s = w1s + WBYTES;
     uint8_t* at = w2s + WBYTES;
-    uint8_t* qb = at + BIG;  // 2 x 16 KB: Q tiles, O staged in place
-    ApplyBars* bars = reinterpret_cast<ApplyBars*>(qb + 2 * TILE);
+    uint8_t* qb = at + BIG;  // NQB x 16 KB: Q tiles, O staged in place
+    ApplyBars* bars = reinterpret_cast<ApplyBars*>(qb + NQB * TILE);
 
     const int split = blockIdx.x, u = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->wfull, 1);
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NQB; ++b) {
             mbar_init(&bars->qfull[b], 1);
             mbar_init(&bars->qfree[b], EPI_WARPS);
         }
@@ -518,8 +519,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             tma_load_weights(w1s, w2s, &tm_w1, &tm_w2, u, &bars->wfull);  // this unit's W1*, W2*
             for (int i = 0; i < ntiles; ++i) {
-                const int b = i & 1;
-                if (i >= 2) mbar_wait(&bars->qfree[b], ((i - 2) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                const int b = i % NQB;
+                if (i >= NQB) mbar_wait(&bars->qfree[b], (i / NQB - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                 mbar_expect_tx(&bars->qfull[b], TILE);
                 tma_load_3d(qb + b * TILE, &tm_q, 0, t0 + i * MT, u, &bars->qfull[b]);
             }
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t IZ = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t IO = tc::idesc_bf16(128, 64, 0, 1);
             auto issue_z = [&](int i, int half) {
-                const uint32_t qa = smem_u32(qb + (i & 1) * TILE);
+                const uint32_t qa = smem_u32(qb + (i % NQB) * TILE);
                 tc::fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
@@ -556,7 +557,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      tc::smem_desc(w2a + ks * 2048, 8192, 1024, 2), IO, ks > 0);
                     if (half) tc::commit(&bars->ofull[ob]);
                     if (i + 1 < ntiles) {
-                        if (half == 0) mbar_wait(&bars->qfull[(i + 1) & 1], ((i + 1) >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                        if (half == 0)
+                            mbar_wait(&bars->qfull[(i + 1) % NQB], ((i + 1) / NQB) & 1, TTT_DEVERR_TIMEOUT_TMA);
                         issue_z(i + 1, half);
                     }
                 }
@@ -566,9 +568,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q4 = warp & 3, ch = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-        for (int i = 0; i < ntiles; ++i) {
-            const int b = i & 1, ob = i & 1;
+        // O of tile j: TMEM -> bf16 over its Q tile (the Z MMAs that read it have completed) -> TMA
+        auto o_store = [&](int j) {
+            const int b = j % NQB, ob = j & 1;
             uint8_t* tile = qb + b * TILE;
+            mbar_wait(&bars->ofull[ob], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            tc::fence_after();
+            {
+                float o[32];
+                ld32(lane_base + COL_O + ob * 64 + ch * 32, o);
+                tc::wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 8) store8_bf16(tile, swz<3>(r * ROWB + (ch * 32 + c) * 2), &o[c]);
+            }
+            tc::fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->oread[ob]);
+            // both column halves of every row quarter are in shared memory once oread completes
+            mbar_wait(&bars->oread[ob], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            if (ch == 0 && lane == 0) {
+                const int row0 = j * MT + q4 * 32;
+                if (row0 < n_valid) {
+                    tma_store_3d(&tm_o, 0, t0 + row0, u, tile + q4 * 32 * ROWB);
+                    tma_store_commit();
+                    tma_store_wait_read_all();
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->qfree[b]);
+        };
+        // gelu of tile i, then the output of tile i - 1 (whose MMAs ran meanwhile)
+        for (int i = 0; i < ntiles; ++i) {
             for (int half = 0; half < 2; ++half) {  // A = gelu(Z), 64 columns per warp and half
                 mbar_wait(half ? &bars->z1full : &bars->z0full, i & 1, TTT_DEVERR_TIMEOUT_PEER);
                 tc::fence_after();
@@ -589,33 +620,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(half ? &bars->a1ready : &bars->a0ready);
             }
-            // O = A W2* -> bf16 over the Q tile (the Z MMAs that read it have completed) -> TMA
-            mbar_wait(&bars->ofull[ob], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
-            {
-                float o[32];
-                ld32(lane_base + COL_O + ob * 64 + ch * 32, o);
-                tc::wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) store8_bf16(tile, swz<3>(r * ROWB + (ch * 32 + j) * 2), &o[j]);
-            }
-            tc::fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->oread[ob]);
-            // both column halves of every row quarter are in shared memory once oread completes
-            mbar_wait(&bars->oread[ob], (i >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-            if (ch == 0 && lane == 0) {
-                const int row0 = i * MT + q4 * 32;
-                if (row0 < n_valid) {
-                    tma_store_3d(&tm_o, 0, t0 + row0, u, tile + q4 * 32 * ROWB);
-                    tma_store_commit();
-                    tma_store_wait_read_all();
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->qfree[b]);
+            if (i >= 1) o_store(i - 1);
         }
+        if (ntiles > 0) o_store(ntiles - 1);
         if (lane == 0) tma_store_wait_all();
     }
     tc::fence_before();

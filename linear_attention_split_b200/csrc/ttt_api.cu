@@ -456,7 +456,7 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
         !tmap_bf16_box(&tw2s, w2b, mlp::D, mlp::HID, U, 64, mlp::HID, sw))
         return TTT_ERR_CUDA;
     const int smem_g = 2 * mlp::WBYTES + 2 * mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::GradBars) + 1024;
-    const int smem_a = 2 * mlp::WBYTES + mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
+    const int smem_a = 2 * mlp::WBYTES + mlp::BIG + mlp::NQB * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
     if (smem_g > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(mlp::grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_g) != cudaSuccess ||
         cudaFuncSetAttribute(mlp::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
