@@ -87,8 +87,8 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
     uint8_t* slots = smem;
     float* partial = reinterpret_cast<float*>(smem + p.nslots * p.slot_bytes);  // [C][9], read by peers
     float* wst = partial + C * NTAP;                                             // [C][9]
-    Bars* bars = reinterpret_cast<Bars*>(wst + C * NTAP);
-    float* red = reinterpret_cast<float*>(slots);  // [cw][9][C], aliases the row slots after use
+    float* red = wst + C * NTAP;                                                 // [cw][9][C]
+    Bars* bars = reinterpret_cast<Bars*>(red + MAX_CW * NTAP * C);
     const int CW = p.cw;
     const int THREADS = (CW + 1) * 32;
 
@@ -178,16 +178,25 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
 #pragma unroll
     for (int t = 0; t < NTAP; ++t) g[t] = make_float2(0.f, 0.f);
 
+    // The 3-row K window lives in registers and slides by one row per output row: each K
+    // row is awaited, read and released (kempty) once; likewise each V row.
+    const uint8_t* kbase = slots + px0 * PXB + c * 2;  // smem pixel px0 = image pixel px0 - 1
+    auto load_krow = [&](int k, float2* dst) {
+        const int s = k % KS;
+        mbar_wait(&bars->kfull[s], (k / KS) & 1, TTT_DEVERR_TIMEOUT_TMA);
+#pragma unroll
+        for (int xi = 0; xi < PXW + 2; ++xi)
+            dst[xi] = bf2(*reinterpret_cast<const uint32_t*>(kbase + s * p.slot_bytes + xi * PXB));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->kempty[s]);  // the row is in registers now
+    };
+    float2 kw[3][PXW + 2];
+    if (rows > 0) {
+        load_krow(0, kw[0]);
+        load_krow(1, kw[1]);
+    }
     for (int j = 0; j < rows; ++j) {
-        float2 kw[3][PXW + 2];
-#pragma unroll
-        for (int dy = 0; dy < 3; ++dy) {
-            const int k = j + dy, s = k % KS;
-            mbar_wait(&bars->kfull[s], (k / KS) & 1, TTT_DEVERR_TIMEOUT_TMA);
-            const uint8_t* base = slot(s) + px0 * PXB + c * 2;  // smem pixel px0 = image px0 - 1
-#pragma unroll
-            for (int xi = 0; xi < PXW + 2; ++xi) kw[dy][xi] = bf2(*reinterpret_cast<const uint32_t*>(base + xi * PXB));
-        }
+        load_krow(j + 2, kw[2]);
         const int vs = j % VS;
         mbar_wait(&bars->vfull[vs], (j / VS) & 1, TTT_DEVERR_TIMEOUT_TMA);
         const uint8_t* vbase = slot(KS + vs) + (px0 + 1) * PXB + c * 2;
@@ -203,13 +212,18 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
             }
         }
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&bars->kempty[j % KS]);  // K row j is not used by later rows
-            mbar_arrive(&bars->vempty[vs]);
+        if (lane == 0) mbar_arrive(&bars->vempty[vs]);
+#pragma unroll
+        for (int xi = 0; xi < PXW + 2; ++xi) {
+            kw[0][xi] = kw[1][xi];
+            kw[1][xi] = kw[2][xi];
         }
     }
-    // ---- per-CTA partial: sum the eight warps' gradients ----------------------------------
-    consumers_sync(CW * 32);  // every warp is done with the row slots
+    // every K/V row has been read: the slots may take the Q rows while the gradients reduce
+    fence_proxy_async_smem();
+    consumers_sync(CW * 32);
+    if (threadIdx.x == 0) mbar_arrive(&bars->qgo);
+    // ---- per-CTA partial: sum the warps' gradients (dedicated buffer) ----------------------
 #pragma unroll
     for (int t = 0; t < NTAP; ++t) {
         red[(warp * NTAP + t) * C + c] = g[t].x;
@@ -218,16 +232,10 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
     consumers_sync(CW * 32);
     for (int e = threadIdx.x; e < C * NTAP; e += CW * 32) {
         const int ch = e / NTAP, t = e % NTAP;
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < CW; ++w) s += red[(w * NTAP + t) * C + ch];
-        partial[e] = s;
+        float sum = 0.f;
+        for (int w = 0; w < CW; ++w) sum += red[(w * NTAP + t) * C + ch];
+        partial[e] = sum;
     }
-    consumers_sync(CW * 32);
-    zero_pads(p.nslots, threadIdx.x, CW * 32);  // the reduction buffer covered some padding
-    fence_proxy_async_smem();  // the slots are written next by TMA (Q)
-    consumers_sync(CW * 32);
-    if (threadIdx.x == 0) mbar_arrive(&bars->qgo);
     cluster_sync_all();
 
     // ---- w* = w0 - (eta/N) sum over the cluster, in rank order ------------------------------
@@ -252,15 +260,20 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
     float2 wf[NTAP];
 #pragma unroll
     for (int t = 0; t < NTAP; ++t) wf[t] = make_float2(wst[c * NTAP + t], wst[(c + 1) * NTAP + t]);
+    const uint8_t* qbase = slots + px0 * PXB + c * 2;
+    auto load_qrow = [&](int k, float2* dst) {  // Q row y0 - 1 + k lives in slot k
+        mbar_wait(&bars->qfull[k], 0, TTT_DEVERR_TIMEOUT_TMA);
+#pragma unroll
+        for (int xi = 0; xi < PXW + 2; ++xi)
+            dst[xi] = bf2(*reinterpret_cast<const uint32_t*>(qbase + k * p.slot_bytes + xi * PXB));
+    };
+    float2 qw[3][PXW + 2];
+    if (rows > 0) {
+        load_qrow(0, qw[0]);
+        load_qrow(1, qw[1]);
+    }
     for (int j = 0; j < rows; ++j) {
-        float2 qw[3][PXW + 2];
-#pragma unroll
-        for (int dy = 0; dy < 3; ++dy) {
-            mbar_wait(&bars->qfull[j + dy], 0, TTT_DEVERR_TIMEOUT_TMA);
-            const uint8_t* base = slot(j + dy) + px0 * PXB + c * 2;
-#pragma unroll
-            for (int xi = 0; xi < PXW + 2; ++xi) qw[dy][xi] = bf2(*reinterpret_cast<const uint32_t*>(base + xi * PXB));
-        }
+        load_qrow(j + 2, qw[2]);
         __nv_bfloat16* orow = p.out + (((size_t)b * p.Hg + y0 + j) * p.Wg) * C + c;
 #pragma unroll
         for (int i = 0; i < PXW; ++i) {
@@ -270,6 +283,11 @@ __global__ void __launch_bounds__((MAX_CW + 1) * 32, 1)
                 for (int t = 0; t < NTAP; ++t) o = ffma2(wf[t], qw[t / 3][i + t % 3], o);
                 *reinterpret_cast<uint32_t*>(orow + (size_t)(px0 + i) * C) = pack_bf16(o.x, o.y);
             }
+        }
+#pragma unroll
+        for (int xi = 0; xi < PXW + 2; ++xi) {
+            qw[0][xi] = qw[1][xi];
+            qw[1][xi] = qw[2][xi];
         }
     }
     cluster_wait_acquire();

@@ -313,7 +313,7 @@ int dwconv_fused(const void* q, const void* k, const void* v, const float* w0, v
     p.Hg = Hg;
     p.Wg = Wg;
     p.eta_over_n = (float)((double)eta / ((double)Hg * Wg));
-    const int smem = p.nslots * p.slot_bytes + 2 * dwc::C * dwc::NTAP * 4 + (int)sizeof(dwc::Bars) + 128;
+    const int smem = p.nslots * p.slot_bytes + (2 + dwc::MAX_CW) * dwc::C * dwc::NTAP * 4 + (int)sizeof(dwc::Bars) + 128;
     if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
     CUtensorMap tk, tv, tq;
     if (!tmap_bf16_rows(&tk, k, dwc::C, Wg, Hg, B) || !tmap_bf16_rows(&tv, v, dwc::C, Wg, Hg, B) ||
