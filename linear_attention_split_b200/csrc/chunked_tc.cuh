@@ -146,6 +146,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     group_sync(dir);
     uint32_t bw[4][2][2];  // B fragments of the current W (bf16)
     load_b(wt_a, bw);
+    // The partner direction's parked partials, read PF steps before they are added (all of
+    // them are written before the barrier at step nc/2), so that the read's latency stays
+    // off the step-to-step chain.
+    constexpr int PF = 2;
+    float2 pre0[4], pre1[4];  // steps of even / odd parity
+    const int rr = 16 * wq + (lane >> 2);
+    auto adds_at = [&](int st) { return st >= nc / 2 && !(2 * st == nc - 1 && dir == 0); };
+    auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st
+        const size_t t0c = (size_t)u * p.N + (size_t)chunk_of(dir, st) * CB;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 x =
+                    *reinterpret_cast<const float2*>(&p.park[(t0c + rr + 8 * h) * D + col0 + nt * 8 + 2 * (lane & 3)]);
+                if (st & 1)
+                    pre1[2 * nt + h] = x;
+                else
+                    pre0[2 * nt + h] = x;
+            }
+    };
 
     for (int step = 0; step < nc; ++step) {
         const int s = step % STAGES;
@@ -236,15 +257,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (park) {
                         *reinterpret_cast<float2*>(&p.park[idx]) = val;
                     } else {
-                        const float2 other = *reinterpret_cast<const float2*>(&p.park[idx]);
+                        const float2 other = (step & 1) ? pre1[2 * nt + h] : pre0[2 * nt + h];
                         *reinterpret_cast<uint32_t*>(&p.out[idx]) = pack_bf16(val.x + other.x, val.y + other.y);
                     }
                 }
             }
         };
         if (first || (middle && dir == 0)) visit(true);
-        if (step == nc / 2) asm volatile("bar.sync 3, 256;" ::: "memory");
+        if (step == nc / 2) {
+            asm volatile("bar.sync 3, 256;" ::: "memory");  // every park is written
+#pragma unroll
+            for (int k = 0; k < PF; ++k)
+                if (step + k < nc && adds_at(step + k)) fetch(step + k);
+        }
         if (!first && !(middle && dir == 0)) visit(false);
+        if (step >= nc / 2 && step + PF < nc && adds_at(step + PF)) fetch(step + PF);  // slot of this step
     }
 }
 
