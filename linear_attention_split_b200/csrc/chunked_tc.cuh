@@ -8,13 +8,20 @@
 //     O_c = Q_c W                      (W after the chunk's update)
 // raster order from W0 and reverse raster order from W0; the layer output is the sum.
 // The output columns of W evolve independently (column j of the update only involves column
-// j of W, V and O), so a CTA owns 16 of the 64 columns and both directions of one unit:
-// warps 0-3 scan forward (chunk s at step s), warps 4-7 backward (chunk nc-1-s at step s),
-// each warp owning 16 tokens of R and O and 16 rows (features) of the W update.  The MMAs
-// are bf16 mma.sync m16n8k16 with fp32 accumulation; W's master copy stays fp32 in
-// registers, and its bf16 copy (the B operand of K_c W and Q_c W) goes through shared memory
-// once per step.  A producer warp streams K_c, Q_c (128B-swizzled) and the CTA's 16 columns
-// of V_c through a TMA ring.  The two directions meet in the middle: at step s < nc/2 each
+// j of W, V and O), so a CTA owns 16 of the 64 columns and both directions of one unit.
+//
+// One recurrence warp per direction (warp 0 forward: chunk s at step s; warp 1 backward:
+// chunk nc-1-s at step s) keeps the whole 64 x 16 slice of W in registers: the fp32 master
+// copy in the m16n8 accumulator layout and its bf16 copy in the B-operand layout of
+// mma.sync m16n8k16.  A step computes R_i = K_i W - V_i for the chunk's four 16-token tiles
+// (32 MMAs), then dW = sum_i K_i^T R_i (32 MMAs).  R_i's accumulators become dW's B operand and
+// W's accumulators the next step's B operand by 8 x 8 transposes in registers (movmatrix);
+// K_i and K_i^T come from the TMA tile by plain and transposing ldmatrix.  Nothing of the
+// recurrence goes through shared memory, and no other warp takes part in it.  The step's K, Q and the CTA's 16 V
+// columns arrive through a TMA ring filled by a producer warp (warp 4).  Each step the
+// recurrence warp hands W's bf16 B fragments (2 KB) to an output warp of its direction
+// (warps 2, 3) through a small ring (wready / wfree); the output warp computes O_c = Q_c W
+// and the combine of the two directions, which meet in the middle: at step s < nc/2 each
 // direction parks its fp32 partial output for its chunk in the workspace; at step s >= nc/2
 // it adds the partner's parked partial, rounds once to bf16 and stores O (deterministic).
 #pragma once
@@ -31,9 +38,11 @@ constexpr int TILE = CB * ROWB;         // 8 KB
 constexpr int VT = CB * NCOL * 2;       // V columns tile: 2 KB
 constexpr int STAGE = 2 * TILE + VT;    // one direction's data for one step
 constexpr int STAGES = 3;
-constexpr int WLD = 24;                 // bf16 row pitch (48 B) of the W and R tiles
-constexpr int WT = D * WLD * 2;         // one 64 x 16 bf16 tile (padded)
-constexpr int THREADS = 9 * 32;         // 8 compute warps + producer
+constexpr int WBUF = 4;                 // depth of the W hand-over ring
+constexpr int WFR = 16 * 32 * 4;        // one W slice as B fragments: 16 registers x 32 lanes
+constexpr int THREADS = 5 * 32;         // 2 recurrence warps, 2 output warps, producer
+constexpr int PF = 2;                   // steps ahead that the partner's partials are copied
+constexpr int PKB = CB * NCOL * 4;       // one chunk's partials for the CTA's columns (4 KB)
 
 struct Params {
     const float* w0;    // [H][64][64]
@@ -44,44 +53,54 @@ struct Params {
 };
 
 struct Bars {
-    uint64_t full[2][STAGES], empty[2][STAGES];
+    uint64_t full[2][STAGES], empty[2][STAGES], wready[2][WBUF], wfree[2][WBUF], pfull[2][PF + 1];
 };
 
-__device__ __forceinline__ void group_sync(int dir) {
-    if (dir == 0)
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-    else
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+// 8 x 8 bf16 transpose across the warp: lane l holds row l/4, columns 2(l%4), 2(l%4)+1 of
+// the input and returns the same positions of the transpose.
+__device__ __forceinline__ uint32_t movt(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
     chunked_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_v16, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_park,
+                   const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;                                    // [dir][stage] {K, Q, V16}
-    uint8_t* wtile = ring + 2 * STAGES * STAGE;              // [dir] W bf16 [64 feats][16 cols]
-    uint8_t* rtile = wtile + 2 * WT;                         // [dir] R bf16 [64 tokens][16 cols]
-    Bars* bars = reinterpret_cast<Bars*>(rtile + 2 * WT);
+    uint8_t* wfr = ring + 2 * STAGES * STAGE;                // [dir][WBUF] W B fragments
+    uint8_t* pkr = wfr + 2 * WBUF * WFR;                     // [dir][PF + 1] parked partials
+    Bars* bars = reinterpret_cast<Bars*>(pkr + 2 * (PF + 1) * PKB);
 
     const int grp = blockIdx.x, u = blockIdx.y;
     const int col0 = grp * NCOL;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;  // fragment row / column-pair of this lane
     const int nc = p.nc;
     auto stage_ptr = [&](int dir, int s) { return ring + (dir * STAGES + s) * STAGE; };
     auto chunk_of = [&](int dir, int step) { return dir == 0 ? step : nc - 1 - step; };
+    auto wfr_ptr = [&](int dir, int b) { return reinterpret_cast<uint4*>(wfr + (dir * WBUF + b) * WFR); };
 
     if (threadIdx.x == 0) {
-        for (int d = 0; d < 2; ++d)
+        for (int d = 0; d < 2; ++d) {
             for (int s = 0; s < STAGES; ++s) {
                 mbar_init(&bars->full[d][s], 1);
-                mbar_init(&bars->empty[d][s], 4);
+                mbar_init(&bars->empty[d][s], 2);  // the direction's recurrence and output warps
             }
+            for (int b = 0; b < WBUF; ++b) {
+                mbar_init(&bars->wready[d][b], 1);
+                mbar_init(&bars->wfree[d][b], 1);
+            }
+            for (int b = 0; b <= PF; ++b) mbar_init(&bars->pfull[d][b], 1);
+        }
         mbar_fence_init();
     }
     __syncthreads();
 
-    if (warp == 8) {
+    if (warp == 4) {
         // ================================ producer ======================================
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
@@ -102,176 +121,245 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
 
-    // =================================== compute warps ===================================
-    const int dir = warp >> 2;          // 0 forward, 1 backward
-    const int wq = warp & 3;            // 16-row block of this warp
-    uint8_t* wt = wtile + dir * WT;
-    uint8_t* rt = rtile + dir * WT;
-    const uint32_t wt_a = smem_u32(wt), rt_a = smem_u32(rt);
+    // A fragments (16 tokens x 16 features, k-step ks) of a 128B-swizzled [token][64] tile
+    auto load_a = [&](uint32_t tile, int i, int ks, uint32_t* a) {
+        const int row = 16 * i + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int chunk = 2 * ks + (lane >> 4);
+        ldsm_x4(tile + swz<3>(row * ROWB + chunk * 16), a[0], a[1], a[2], a[3]);
+    };
 
-    // master W rows [16 wq, 16 wq + 16) x my 16 columns, C-fragment layout of m16n8
-    float wm[2][4];
-    {
-        const float* W0 = p.w0 + (size_t)(u % p.H) * D * D;
-        const int r = 16 * wq + (lane >> 2);
+    if (warp < 2) {
+        // ============================ recurrence warps ==================================
+        const int dir = warp;
+        // W rows (features) 16 mt + g (+8), columns 8 j + 2t (+1) of this CTA's slice
+        float wm[4][2][4];
+        {
+            const float* W0 = p.w0 + (size_t)(u % p.H) * D * D + col0;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int cj = col0 + nt * 8 + 2 * (lane & 3);
-            wm[nt][0] = W0[r * D + cj];
-            wm[nt][1] = W0[r * D + cj + 1];
-            wm[nt][2] = W0[(r + 8) * D + cj];
-            wm[nt][3] = W0[(r + 8) * D + cj + 1];
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = 16 * mt + g, cj = 8 * j + 2 * t;
+                    wm[mt][j][0] = W0[r * D + cj];
+                    wm[mt][j][1] = W0[r * D + cj + 1];
+                    wm[mt][j][2] = W0[(r + 8) * D + cj];
+                    wm[mt][j][3] = W0[(r + 8) * D + cj + 1];
+                }
         }
-    }
-    // publish W rows as bf16 [feature][col] (pitch 48 B)
-    auto publish = [&](uint8_t* tile, const float (*v)[4], int rbase) {
-        const int r = rbase + (lane >> 2);
+        // bf16 W as B fragments: k-step mt (features 16 mt..), n-tile j (columns 8 j..)
+        uint32_t bw[4][2][2];
+        auto make_b = [&]() {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int cj = nt * 8 + 2 * (lane & 3);
-            *reinterpret_cast<uint32_t*>(tile + (r * WLD + cj) * 2) = pack_bf16(v[nt][0], v[nt][1]);
-            *reinterpret_cast<uint32_t*>(tile + ((r + 8) * WLD + cj) * 2) = pack_bf16(v[nt][2], v[nt][3]);
-        }
-    };
-    // B fragments (k = rows of a [64][16] bf16 tile, n = 16 columns) for four k-steps
-    auto load_b = [&](uint32_t base, uint32_t (*b)[2][2]) {
+            for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const int row = ks * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-            const int colb = (lane >> 4) * 16;  // bytes: columns 0-7 or 8-15
-            ldsm_x4_t(base + row * WLD * 2 + colb, b[ks][0][0], b[ks][0][1], b[ks][1][0], b[ks][1][1]);
-        }
-    };
-    publish(wt, wm, 16 * wq);
-    group_sync(dir);
-    uint32_t bw[4][2][2];  // B fragments of the current W (bf16)
-    load_b(wt_a, bw);
-    // The partner direction's parked partials, read PF steps before they are added (all of
-    // them are written before the barrier at step nc/2), so that the read's latency stays
-    // off the step-to-step chain.
-    constexpr int PF = 2;
-    float2 pre0[4], pre1[4];  // steps of even / odd parity
-    const int rr = 16 * wq + (lane >> 2);
-    auto adds_at = [&](int st) { return st >= nc / 2 && !(2 * st == nc - 1 && dir == 0); };
-    auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st
-        const size_t t0c = (size_t)u * p.N + (size_t)chunk_of(dir, st) * CB;
+                for (int j = 0; j < 2; ++j) {
+                    bw[mt][j][0] = movt(pack_bf16(wm[mt][j][0], wm[mt][j][1]));
+                    bw[mt][j][1] = movt(pack_bf16(wm[mt][j][2], wm[mt][j][3]));
+                }
+        };
+        make_b();
+        // A step issues the R MMAs of all four token tiles (k-steps outermost, so that eight
+        // independent accumulators separate two dependent MMAs), then the dW MMAs tile by
+        // tile; the tensor pipe stays busy while each tile's R drains into dW's operand.
+        uint32_t ka[4][4][4];  // K_i A fragments: [tile i][k-step ks] (tokens 16 i.., features 16 ks..)
+        mbar_wait(&bars->full[dir][0], 0, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float2 x =
-                    *reinterpret_cast<const float2*>(&p.park[(t0c + rr + 8 * h) * D + col0 + nt * 8 + 2 * (lane & 3)]);
-                if (st & 1)
-                    pre1[2 * nt + h] = x;
-                else
-                    pre0[2 * nt + h] = x;
+            for (int ks = 0; ks < 4; ++ks) load_a(smem_u32(stage_ptr(dir, 0)), i, ks, ka[i][ks]);
+        for (int step = 0; step < nc; ++step) {
+            const int s = step % STAGES;
+            uint8_t* st = stage_ptr(dir, s);
+            const uint32_t kb = smem_u32(st);
+            const uint8_t* vt = st + 2 * TILE;
+            // ---- R_i = K_i W for the four tiles ---------------------------------------------
+            float r[4][2][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) r[i][j][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) mma_bf16(r[i][j], ka[i][ks], bw[ks][j][0], bw[ks][j][1]);
+            // K_i^T as A fragments (features 16 mt.., tokens 16 i..): transposing loads
+            uint32_t kt[4][4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt) {
+                    const int row = 16 * i + (lane >> 4) * 8 + (lane & 7);
+                    const int chunk = 2 * mt + ((lane >> 3) & 1);
+                    ldsm_x4_t(kb + swz<3>(row * ROWB + chunk * 16), kt[i][mt][0], kt[i][mt][1], kt[i][mt][2], kt[i][mt][3]);
+                }
+            // ---- dW = sum_i K_i^T (R_i - V_i) -------------------------------------------------
+            float dw[4][2][4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dw[mt][j][e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // R_i - V_i as the B operand of dW (k = tokens 16 i.., n = columns 8 j..)
+                uint32_t rb[2][2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int cj = 8 * j + 2 * t;
+                    const float2 v0 = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g) * NCOL + cj) * 2));
+                    const float2 v1 = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g + 8) * NCOL + cj) * 2));
+                    rb[j][0] = movt(pack_bf16(r[i][j][0] - v0.x, r[i][j][1] - v0.y));
+                    rb[j][1] = movt(pack_bf16(r[i][j][2] - v1.x, r[i][j][3] - v1.y));
+                }
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) mma_bf16(dw[mt][j], kt[i][mt], rb[j][0], rb[j][1]);
             }
-    };
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, V of this step consumed
+            // the next step's tile and a free hand-over slot, tested together; the next
+            // step's K fragments load while this step's dW drains
+            const int b = step % WBUF, use = step / WBUF;
+            const int sn = (step + 1) % STAGES;
+            const bool nf = step + 1 >= nc || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
+            const bool wf = use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
+            if (step + 1 < nc) {
+                if (!nf) mbar_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) load_a(smem_u32(stage_ptr(dir, sn)), i, ks, ka[i][ks]);
+            }
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) wm[mt][j][e] -= p.eta_over_b * dw[mt][j][e];
+            make_b();
+            // ---- hand W (after this step) to the output warp -----------------------------
+            if (!wf) mbar_wait(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            {
+                uint4* dst = wfr_ptr(dir, b);
+                const uint32_t* f = &bw[0][0][0];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    dst[q * 32 + lane] = make_uint4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->wready[dir][b]);
+        }
+        return;
+    }
 
+    // ================================= output warps ========================================
+    // O_c = Q_c W (W after the chunk's update) for the chunk's 64 tokens x 16 columns, then
+    // the combine: chunk c is visited by the forward direction at step c and by the backward
+    // direction at step nc-1-c; the first visit parks its fp32 partial, the second adds it.
+    // For odd nc both visit the middle chunk at the same step: the forward warp parks, then
+    // the backward warp adds.  One barrier over the two output warps at step nc/2 orders all
+    // parks before all additions.  The partner's parked partials (64 tokens x 16 columns,
+    // fp32) are fetched PF steps ahead by one TMA box each into a ring of PF + 1 slots.
+    const int dir = warp - 2;
+    uint8_t* pk = pkr + dir * (PF + 1) * PKB;
+    const int a0 = (nc & 1) && dir == 0 ? nc / 2 + 1 : nc / 2;  // first step that adds
+    auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st
+        if (lane == 0 && st < nc && st >= a0) {
+            const int sl = (st - a0) % (PF + 1);
+            mbar_expect_tx(&bars->pfull[dir][sl], PKB);
+            tma_load_3d(pk + sl * PKB, &tm_park, col0, chunk_of(dir, st) * CB, u, &bars->pfull[dir][sl]);
+        }
+    };
     for (int step = 0; step < nc; ++step) {
         const int s = step % STAGES;
+        const int b = step % WBUF, use = step / WBUF;
         mbar_wait(&bars->full[dir][s], (step / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
-        const int c = chunk_of(dir, step);
-        uint8_t* st = stage_ptr(dir, s);
-        const uint32_t kb = smem_u32(st), qb = kb + TILE;
-        const uint8_t* vt = st + 2 * TILE;
-
-        // ---- R = K_c W - V_c for tokens [16 wq, +16) -------------------------------------
-        float acc[2][4] = {};
+        const uint32_t qb = smem_u32(stage_ptr(dir, s)) + TILE;
+        uint32_t qa[4][4];
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a[4];
-            const int row = 16 * wq + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int chunk = 2 * ks + (lane >> 4);
-            ldsm_x4(kb + swz<3>(row * ROWB + chunk * 16), a[0], a[1], a[2], a[3]);
-            mma_bf16(acc[0], a, bw[ks][0][0], bw[ks][0][1]);
-            mma_bf16(acc[1], a, bw[ks][1][0], bw[ks][1][1]);
-        }
+        for (int ks = 0; ks < 4; ++ks) load_a(qb, 0, ks, qa[ks]);
+        mbar_wait(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
+        uint32_t bw[4][2][2];
         {
-            const int r = 16 * wq + (lane >> 2);
+            const uint4* src = wfr_ptr(dir, b);
+            uint32_t* f = &bw[0][0][0];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int cj = nt * 8 + 2 * (lane & 3);
-                const float2 v0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vt + (r * NCOL + cj) * 2));
-                const float2 v1 =
-                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vt + ((r + 8) * NCOL + cj) * 2));
-                acc[nt][0] -= v0.x;
-                acc[nt][1] -= v0.y;
-                acc[nt][2] -= v1.x;
-                acc[nt][3] -= v1.y;
+            for (int q = 0; q < 4; ++q) {
+                const uint4 x = src[q * 32 + lane];
+                f[4 * q] = x.x;
+                f[4 * q + 1] = x.y;
+                f[4 * q + 2] = x.z;
+                f[4 * q + 3] = x.w;
             }
-        }
-        publish(rt, acc, 16 * wq);
-        group_sync(dir);  // R complete; every warp has read W for this step
-        // ---- W rows [16 wq, +16) -= (eta/b) K_c^T R ---------------------------------------
-        uint32_t br[4][2][2];
-        load_b(rt_a, br);
-        float dw[2][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {  // k = tokens 16 ks..
-            uint32_t a[4];
-            const int row = ks * 16 + (lane >> 4) * 8 + (lane & 7);
-            const int chunk = wq * 2 + ((lane >> 3) & 1);
-            ldsm_x4_t(kb + swz<3>(row * ROWB + chunk * 16), a[0], a[1], a[2], a[3]);
-            mma_bf16(dw[0], a, br[ks][0][0], br[ks][0][1]);
-            mma_bf16(dw[1], a, br[ks][1][0], br[ks][1][1]);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) wm[nt][e] -= p.eta_over_b * dw[nt][e];
-        publish(wt, wm, 16 * wq);  // every warp read the old W before the barrier above
-        group_sync(dir);  // new W tile complete
-        // ---- O_c = Q_c W for tokens [16 wq, +16) ------------------------------------------
-        load_b(wt_a, bw);
-        float o[2][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a[4];
-            const int row = 16 * wq + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int chunk = 2 * ks + (lane >> 4);
-            ldsm_x4(qb + swz<3>(row * ROWB + chunk * 16), a[0], a[1], a[2], a[3]);
-            mma_bf16(o[0], a, bw[ks][0][0], bw[ks][0][1]);
-            mma_bf16(o[1], a, bw[ks][1][0], bw[ks][1][1]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, Q, V of this step consumed
-        // ---- combine the two directions ---------------------------------------------------
-        // chunk c is visited by the forward warps at step c and by the backward warps at step
-        // nc-1-c: the first visit parks its partial, the second adds it.  For odd nc both
-        // visit the middle chunk at the same step: the forward warps park, then the backward
-        // warps add.  One barrier over the compute warps at step nc/2 orders all parks
-        // before all additions.
-        const int r = 16 * wq + (lane >> 2);
-        const size_t tok0 = (size_t)u * p.N + (size_t)c * CB;
-        const bool first = 2 * step < nc - 1;
-        const bool middle = 2 * step == nc - 1;
-        auto visit = [&](bool park) {
+        if (lane == 0) mbar_arrive(&bars->wfree[dir][b]);
+        float o[4][2][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int cj = col0 + nt * 8 + 2 * (lane & 3);
+        for (int i = 0; i < 4; ++i) {
+            uint32_t qn[4][4];
+            if (i < 3) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const size_t idx = (tok0 + r + 8 * h) * D + cj;
-                    const float2 val = make_float2(o[nt][2 * h], o[nt][2 * h + 1]);
-                    if (park) {
-                        *reinterpret_cast<float2*>(&p.park[idx]) = val;
-                    } else {
-                        const float2 other = (step & 1) ? pre1[2 * nt + h] : pre0[2 * nt + h];
-                        *reinterpret_cast<uint32_t*>(&p.out[idx]) = pack_bf16(val.x + other.x, val.y + other.y);
-                    }
-                }
+                for (int ks = 0; ks < 4; ++ks) load_a(qb, i + 1, ks, qn[ks]);
             }
-        };
-        if (first || (middle && dir == 0)) visit(true);
-        if (step == nc / 2) {
-            asm volatile("bar.sync 3, 256;" ::: "memory");  // every park is written
 #pragma unroll
-            for (int k = 0; k < PF; ++k)
-                if (step + k < nc && adds_at(step + k)) fetch(step + k);
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[i][j][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) mma_bf16(o[i][j], qa[ks], bw[ks][j][0], bw[ks][j][1]);
+            if (i < 3) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) qa[ks][e] = qn[ks][e];
+            }
         }
-        if (!first && !(middle && dir == 0)) visit(false);
-        if (step >= nc / 2 && step + PF < nc && adds_at(step + PF)) fetch(step + PF);  // slot of this step
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // Q of this step consumed
+        const size_t tok0 = (size_t)u * p.N + (size_t)chunk_of(dir, step) * CB;
+        auto visit = [&](bool park) {
+            const float* other = reinterpret_cast<const float*>(pk + ((step - a0) % (PF + 1)) * PKB);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const size_t idx = (tok0 + 16 * i + g + 8 * h) * D + col0 + 8 * j + 2 * t;
+                        const float2 val = make_float2(o[i][j][2 * h], o[i][j][2 * h + 1]);
+                        if (park) {
+                            *reinterpret_cast<float2*>(&p.park[idx]) = val;
+                        } else {
+                            const float2 x = *reinterpret_cast<const float2*>(other + (16 * i + g + 8 * h) * NCOL + 8 * j + 2 * t);
+                            *reinterpret_cast<uint32_t*>(&p.out[idx]) = pack_bf16(val.x + x.x, val.y + x.y);
+                        }
+                    }
+        };
+        if (step < a0) visit(true);
+        if (step == nc / 2) {
+            // every park is written, and visible to the tensor-copy reads that follow
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            asm volatile("bar.sync 1, 64;" ::: "memory");
+#pragma unroll
+            for (int k = 0; k < PF; ++k) fetch(a0 + k);
+        }
+        if (step >= a0) {
+            mbar_wait(&bars->pfull[dir][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1, TTT_DEVERR_TIMEOUT_TMA);
+            visit(false);
+            __syncwarp();  // every lane has read the slot before it is refilled
+            fetch(step + PF);
+        }
     }
 }
 

@@ -510,9 +510,10 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
     p.N = N;
     p.nc = N / chk::CB;
     p.eta_over_b = (float)((double)eta / (double)chk::CB);
-    const int smem = 2 * chk::STAGES * chk::STAGE + 2 * 2 * chk::WT + (int)sizeof(chk::Bars) + 1024;
+    const int smem = 2 * chk::STAGES * chk::STAGE + 2 * chk::WBUF * chk::WFR + 2 * (chk::PF + 1) * chk::PKB +
+                     (int)sizeof(chk::Bars) + 1024;
     if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
-    CUtensorMap tk, tq, tv;
+    CUtensorMap tk, tq, tv, tp;
     if (!tmap_bf16_3d(&tk, k, 64, N, U, chk::CB, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !tmap_bf16_3d(&tq, q, 64, N, U, chk::CB, CU_TENSOR_MAP_SWIZZLE_128B))
         return TTT_ERR_CUDA;
@@ -527,11 +528,17 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return TTT_ERR_CUDA;
+        // parked partials (fp32 [U][N][64]): box of 16 columns x 64 tokens, no swizzle
+        cuuint64_t pstrides[2] = {256, (cuuint64_t)N * 256};
+        if (fn(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws, dims, pstrides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return TTT_ERR_CUDA;
     }
     auto kern = chk::chunked_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return TTT_ERR_CUDA;
-    kern<<<dim3(chk::GROUPS, U), chk::THREADS, smem, st>>>(tk, tq, tv, p);
+    kern<<<dim3(chk::GROUPS, U), chk::THREADS, smem, st>>>(tk, tq, tv, tp, p);
     return launched(1);
 }
 
