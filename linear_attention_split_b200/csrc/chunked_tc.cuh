@@ -186,6 +186,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) mma_bf16(r[i][j], ka[i][ks], bw[ks][j][0], bw[ks][j][1]);
+            // the next step's tile and a free hand-over slot, tested now so that the tests'
+            // latency passes under the dW work
+            const int b = step % WBUF, use = step / WBUF;
+            const int sn = (step + 1) % STAGES;
+            const bool nf = step + 1 >= nc || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
+            const bool wf = use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
             // K_i^T as A fragments (features 16 mt.., tokens 16 i..): transposing loads
             uint32_t kt[4][4][4];
 #pragma unroll
@@ -204,10 +210,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) dw[mt][j][e] = 0.f;
+            // R_i - V_i as the B operand of dW (k = tokens 16 i.., n = columns 8 j..)
+            uint32_t rb[4][2][2];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                // R_i - V_i as the B operand of dW (k = tokens 16 i.., n = columns 8 j..)
-                uint32_t rb[2][2];
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int cj = 8 * j + 2 * t;
@@ -215,22 +221,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                         *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g) * NCOL + cj) * 2));
                     const float2 v1 = __bfloat1622float2(
                         *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g + 8) * NCOL + cj) * 2));
-                    rb[j][0] = movt(pack_bf16(r[i][j][0] - v0.x, r[i][j][1] - v0.y));
-                    rb[j][1] = movt(pack_bf16(r[i][j][2] - v1.x, r[i][j][3] - v1.y));
+                    rb[i][j][0] = movt(pack_bf16(r[i][j][0] - v0.x, r[i][j][1] - v0.y));
+                    rb[i][j][1] = movt(pack_bf16(r[i][j][2] - v1.x, r[i][j][3] - v1.y));
                 }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) mma_bf16(dw[mt][j], kt[i][mt], rb[j][0], rb[j][1]);
-            }
+                    for (int j = 0; j < 2; ++j) mma_bf16(dw[mt][j], kt[i][mt], rb[i][j][0], rb[i][j][1]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, V of this step consumed
-            // the next step's tile and a free hand-over slot, tested together; the next
-            // step's K fragments load while this step's dW drains
-            const int b = step % WBUF, use = step / WBUF;
-            const int sn = (step + 1) % STAGES;
-            const bool nf = step + 1 >= nc || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
-            const bool wf = use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
+            // the next step's K fragments load while this step's dW drains
             if (step + 1 < nc) {
                 if (!nf) mbar_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
@@ -328,25 +331,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // Q of this step consumed
         const size_t tok0 = (size_t)u * p.N + (size_t)chunk_of(dir, step) * CB;
-        auto visit = [&](bool park) {
-            const float* other = reinterpret_cast<const float*>(pk + ((step - a0) % (PF + 1)) * PKB);
+        auto out_index = [&](int i, int j, int h) {
+            return (tok0 + 16 * i + g + 8 * h) * D + col0 + 8 * j + 2 * t;
+        };
+        if (step < a0) {  // first visit: park the fp32 partial
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const size_t idx = (tok0 + 16 * i + g + 8 * h) * D + col0 + 8 * j + 2 * t;
-                        const float2 val = make_float2(o[i][j][2 * h], o[i][j][2 * h + 1]);
-                        if (park) {
-                            *reinterpret_cast<float2*>(&p.park[idx]) = val;
-                        } else {
-                            const float2 x = *reinterpret_cast<const float2*>(other + (16 * i + g + 8 * h) * NCOL + 8 * j + 2 * t);
-                            *reinterpret_cast<uint32_t*>(&p.out[idx]) = pack_bf16(val.x + x.x, val.y + x.y);
-                        }
-                    }
-        };
-        if (step < a0) visit(true);
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<float2*>(&p.park[out_index(i, j, h)]) =
+                            make_float2(o[i][j][2 * h], o[i][j][2 * h + 1]);
+        }
         if (step == nc / 2) {
             // every park is written, and visible to the tensor-copy reads that follow
             asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -355,8 +352,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int k = 0; k < PF; ++k) fetch(a0 + k);
         }
         if (step >= a0) {
+            // second visit: add the partner's partial, round once, store O.  Every read of the
+            // slot is issued before the first store, so that no read waits behind a store.
             mbar_wait(&bars->pfull[dir][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1, TTT_DEVERR_TIMEOUT_TMA);
-            visit(false);
+            const float* other = reinterpret_cast<const float*>(pk + ((step - a0) % (PF + 1)) * PKB);
+            float2 x[4][2][2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        x[i][j][h] = *reinterpret_cast<const float2*>(other + (16 * i + g + 8 * h) * NCOL + 8 * j + 2 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<uint32_t*>(&p.out[out_index(i, j, h)]) =
+                            pack_bf16(o[i][j][2 * h] + x[i][j][h].x, o[i][j][2 * h + 1] + x[i][j][h].y);
             __syncwarp();  // every lane has read the slot before it is refilled
             fetch(step + PF);
         }
