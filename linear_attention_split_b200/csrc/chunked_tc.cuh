@@ -11,13 +11,14 @@
 // j of W, V and O), so a CTA owns 16 of the 64 columns and both directions of one unit.
 //
 // One recurrence warp per direction (warp 0 forward: chunk s at step s; warp 1 backward:
-// chunk nc-1-s at step s) keeps the whole 64 x 16 slice of W in registers: the fp32 master
-// copy in the m16n8 accumulator layout and its bf16 copy in the B-operand layout of
-// mma.sync m16n8k16.  A step computes R_i = K_i W - V_i for the chunk's four 16-token tiles
-// (32 MMAs), then dW = sum_i K_i^T R_i (32 MMAs).  R_i's accumulators become dW's B operand and
-// W's accumulators the next step's B operand by 8 x 8 transposes in registers (movmatrix);
-// K_i and K_i^T come from the TMA tile by plain and transposing ldmatrix.  Nothing of the
-// recurrence goes through shared memory, and no other warp takes part in it.  The step's K, Q and the CTA's 16 V
+// chunk nc-1-s at step s) keeps the whole 64 x 16 slice of W in registers, as its transpose:
+// the fp32 master copy of W^T in the m16n8 accumulator layout of mma.sync m16n8k16, and its
+// bf16 copy as A fragments.  A step computes R_i^T = W^T K_i^T - V_i^T for the chunk's four
+// 16-token tiles (32 MMAs), then dW^T = sum_i R_i^T K_i (32 MMAs).  In this orientation each
+// accumulator, packed to bf16 pairs, already is the next product's operand (R_i^T's for dW^T,
+// W^T's for the next step's R^T and for Q W); K_i, K_i^T and V_i^T come from the TMA tiles by
+// plain and transposing ldmatrix.  Nothing of the recurrence goes through shared memory, and
+// no other warp takes part in it.  The step's K, Q and the CTA's 16 V
 // columns arrive through a TMA ring filled by a producer warp (warp 4).  Each step the
 // recurrence warp hands W's bf16 B fragments (2 KB) to an output warp of its direction
 // (warps 2, 3) through a small ring (wready / wfree); the output warp computes O_c = Q_c W
@@ -55,14 +56,6 @@ struct Params {
 struct Bars {
     uint64_t full[2][STAGES], empty[2][STAGES], wready[2][WBUF], wfree[2][WBUF], pfull[2][PF + 1];
 };
-
-// 8 x 8 bf16 transpose across the warp: lane l holds row l/4, columns 2(l%4), 2(l%4)+1 of
-// the input and returns the same positions of the transpose.
-__device__ __forceinline__ uint32_t movt(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
 
 __global__ void __launch_bounds__(THREADS, 1)
     chunked_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -130,38 +123,42 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp < 2) {
         // ============================ recurrence warps ==================================
+        // The warp works on transposes, so that every accumulator is already in the layout of
+        // the next product's operand: R_i^T = W^T K_i^T - V_i^T and dW^T = sum_i R_i^T K_i.
+        // Master copy: W^T (16 columns x 64 features) in the m16n8 accumulator layout, n-tile n
+        // = features 8 n..: wt[n] = {W[8n+2t][g], W[8n+2t+1][g], W[8n+2t][8+g], W[8n+2t+1][8+g]}
+        // (column indices relative to this CTA's slice).
         const int dir = warp;
-        // W rows (features) 16 mt + g (+8), columns 8 j + 2t (+1) of this CTA's slice
-        float wm[4][2][4];
+        float wt[8][4];
         {
             const float* W0 = p.w0 + (size_t)(u % p.H) * D * D + col0;
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int r = 16 * mt + g, cj = 8 * j + 2 * t;
-                    wm[mt][j][0] = W0[r * D + cj];
-                    wm[mt][j][1] = W0[r * D + cj + 1];
-                    wm[mt][j][2] = W0[(r + 8) * D + cj];
-                    wm[mt][j][3] = W0[(r + 8) * D + cj + 1];
-                }
+            for (int n = 0; n < 8; ++n) {
+                const int f = 8 * n + 2 * t;
+                wt[n][0] = W0[f * D + g];
+                wt[n][1] = W0[(f + 1) * D + g];
+                wt[n][2] = W0[f * D + 8 + g];
+                wt[n][3] = W0[(f + 1) * D + 8 + g];
+            }
         }
-        // bf16 W as B fragments: k-step mt (features 16 mt..), n-tile j (columns 8 j..)
-        uint32_t bw[4][2][2];
-        auto make_b = [&]() {
+        // bf16 W^T as A fragments, k-step ks = features 16 ks..: pairs of the accumulators.
+        // The same registers are the B fragments of W for O = Q W: (ks, column tile j) takes
+        // {wa[ks][j], wa[ks][2 + j]}.
+        uint32_t wa[4][4];
+        auto make_a = [&]() {
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    bw[mt][j][0] = movt(pack_bf16(wm[mt][j][0], wm[mt][j][1]));
-                    bw[mt][j][1] = movt(pack_bf16(wm[mt][j][2], wm[mt][j][3]));
-                }
+            for (int ks = 0; ks < 4; ++ks) {
+                wa[ks][0] = pack_bf16(wt[2 * ks][0], wt[2 * ks][1]);
+                wa[ks][1] = pack_bf16(wt[2 * ks][2], wt[2 * ks][3]);
+                wa[ks][2] = pack_bf16(wt[2 * ks + 1][0], wt[2 * ks + 1][1]);
+                wa[ks][3] = pack_bf16(wt[2 * ks + 1][2], wt[2 * ks + 1][3]);
+            }
         };
-        make_b();
-        // A step issues the R MMAs of all four token tiles (k-steps outermost, so that eight
-        // independent accumulators separate two dependent MMAs), then the dW MMAs tile by
-        // tile; the tensor pipe stays busy while each tile's R drains into dW's operand.
-        uint32_t ka[4][4][4];  // K_i A fragments: [tile i][k-step ks] (tokens 16 i.., features 16 ks..)
+        make_a();
+        // K_i fragments (ldmatrix of the [token][feature] tile, tokens 16 i.., features
+        // 16 ks..): registers {0, 2} / {1, 3} are the B fragments of K_i^T for tokens
+        // 16 i + 0..7 / 16 i + 8..15.
+        uint32_t ka[4][4][4];
         mbar_wait(&bars->full[dir][0], 0, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -171,28 +168,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int s = step % STAGES;
             uint8_t* st = stage_ptr(dir, s);
             const uint32_t kb = smem_u32(st);
-            const uint8_t* vt = st + 2 * TILE;
-            // ---- R_i = K_i W for the four tiles ---------------------------------------------
-            float r[4][2][4];
+            const uint32_t vb = kb + 2 * TILE;
+            // ---- R_i^T = W^T K_i^T for the four tiles (k-steps outermost) ------------------
+            float rt[4][2][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
+                for (int nn = 0; nn < 2; ++nn)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) r[i][j][e] = 0.f;
+                    for (int e = 0; e < 4; ++e) rt[i][nn][e] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) mma_bf16(r[i][j], ka[i][ks], bw[ks][j][0], bw[ks][j][1]);
+                    for (int nn = 0; nn < 2; ++nn) mma_bf16(rt[i][nn], wa[ks], ka[i][ks][nn], ka[i][ks][2 + nn]);
             // the next step's tile and a free hand-over slot, tested now so that the tests'
             // latency passes under the dW work
             const int b = step % WBUF, use = step / WBUF;
             const int sn = (step + 1) % STAGES;
             const bool nf = step + 1 >= nc || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
             const bool wf = use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
-            // K_i^T as A fragments (features 16 mt.., tokens 16 i..): transposing loads
+            // K_i as B fragments of dW^T (k = tokens 16 i.., n = features): transposing loads;
+            // (features 16 mt + 0..7) takes {kt[i][mt][0], [2]}, (16 mt + 8..15) {[1], [3]}
             uint32_t kt[4][4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -200,37 +198,39 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int mt = 0; mt < 4; ++mt) {
                     const int row = 16 * i + (lane >> 4) * 8 + (lane & 7);
                     const int chunk = 2 * mt + ((lane >> 3) & 1);
-                    ldsm_x4_t(kb + swz<3>(row * ROWB + chunk * 16), kt[i][mt][0], kt[i][mt][1], kt[i][mt][2], kt[i][mt][3]);
+                    ldsm_x4_t(kb + swz<3>(row * ROWB + chunk * 16), kt[i][mt][0], kt[i][mt][1], kt[i][mt][2],
+                              kt[i][mt][3]);
                 }
-            // ---- dW = sum_i K_i^T (R_i - V_i) -------------------------------------------------
-            float dw[4][2][4];
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dw[mt][j][e] = 0.f;
-            // R_i - V_i as the B operand of dW (k = tokens 16 i.., n = columns 8 j..)
-            uint32_t rb[4][2][2];
+            // R_i^T - V_i^T as the A fragments of dW^T (rows = columns, k = tokens 16 i..).
+            // V_i^T comes from a transposing load of the [token][16 column] V tile: matrices
+            // (tokens +0..7 | +8..15) x (columns 0..7 | 8..15).
+            uint32_t ra[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
+                uint32_t vr[4];
+                const int vrow = 16 * i + ((lane >> 4) & 1) * 8 + (lane & 7);
+                ldsm_x4_t(vb + vrow * (NCOL * 2) + ((lane >> 3) & 1) * 16, vr[0], vr[1], vr[2], vr[3]);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int cj = 8 * j + 2 * t;
-                    const float2 v0 = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g) * NCOL + cj) * 2));
-                    const float2 v1 = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162*>(vt + ((16 * i + g + 8) * NCOL + cj) * 2));
-                    rb[i][j][0] = movt(pack_bf16(r[i][j][0] - v0.x, r[i][j][1] - v0.y));
-                    rb[i][j][1] = movt(pack_bf16(r[i][j][2] - v1.x, r[i][j][3] - v1.y));
+                for (int q = 0; q < 4; ++q) {  // q = 2 nn + (rows 8..15)
+                    const int nn = q >> 1, hi = q & 1;
+                    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vr[2 * nn + hi]));
+                    // A fragment order: {rows 0-7, k 0-7}, {rows 8-15, k 0-7}, {rows 0-7, k 8-15}, ...
+                    ra[i][2 * nn + hi] = pack_bf16(rt[i][nn][2 * hi] - v.x, rt[i][nn][2 * hi + 1] - v.y);
                 }
             }
+            // ---- dW^T = sum_i R_i^T K_i (n-tiles of 8 features) -------------------------------
+            float dwt[8][4];
+#pragma unroll
+            for (int n = 0; n < 8; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dwt[n][e] = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) mma_bf16(dw[mt][j], kt[i][mt], rb[i][j][0], rb[i][j][1]);
+                for (int mt = 0; mt < 4; ++mt) {
+                    mma_bf16(dwt[2 * mt], ra[i], kt[i][mt][0], kt[i][mt][2]);
+                    mma_bf16(dwt[2 * mt + 1], ra[i], kt[i][mt][1], kt[i][mt][3]);
+                }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, V of this step consumed
             // the next step's K fragments load while this step's dW drains
@@ -242,20 +242,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int ks = 0; ks < 4; ++ks) load_a(smem_u32(stage_ptr(dir, sn)), i, ks, ka[i][ks]);
             }
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
+            for (int n = 0; n < 8; ++n)
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) wm[mt][j][e] -= p.eta_over_b * dw[mt][j][e];
-            make_b();
+                for (int e = 0; e < 4; ++e) wt[n][e] -= p.eta_over_b * dwt[n][e];
+            make_a();
             // ---- hand W (after this step) to the output warp -----------------------------
             if (!wf) mbar_wait(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             {
                 uint4* dst = wfr_ptr(dir, b);
-                const uint32_t* f = &bw[0][0][0];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[q * 32 + lane] = make_uint4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+                for (int ks = 0; ks < 4; ++ks)
+                    dst[ks * 32 + lane] = make_uint4(wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->wready[dir][b]);
@@ -290,17 +287,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) load_a(qb, 0, ks, qa[ks]);
         mbar_wait(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
-        uint32_t bw[4][2][2];
+        uint32_t bw[4][2][2];  // B fragments of W: k-step ks, column tile j
         {
             const uint4* src = wfr_ptr(dir, b);
-            uint32_t* f = &bw[0][0][0];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 x = src[q * 32 + lane];
-                f[4 * q] = x.x;
-                f[4 * q + 1] = x.y;
-                f[4 * q + 2] = x.z;
-                f[4 * q + 3] = x.w;
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint4 x = src[ks * 32 + lane];
+                bw[ks][0][0] = x.x;
+                bw[ks][1][0] = x.y;
+                bw[ks][0][1] = x.z;
+                bw[ks][1][1] = x.w;
             }
         }
         __syncwarp();
