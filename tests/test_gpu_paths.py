@@ -105,7 +105,7 @@ def test_chunked_80x80_bf16_full():
     check_chunked(8, 3, 6400, 64, 64, "bf16")
 
 
-@pytest.mark.parametrize("N,chunk", [(64, 64), (192, 64), (256, 16), (128, 32), (48, 1), (320, 320)])
+@pytest.mark.parametrize("N,chunk", [(64, 64), (128, 64), (192, 64), (640, 64), (256, 16), (128, 32), (48, 1), (320, 320)])
 def test_chunked_shapes(N, chunk):
     check_chunked(2, 2, N, 64, chunk, "bf16", seed=N + chunk)
 
