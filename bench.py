@@ -99,6 +99,16 @@ def max_over_ranks(pg, x, device):
     return float(t.item())
 
 
+def rank_seed(rank):
+    """Seed of a rank's synthetic inputs: every rank draws its own batch (weak scaling)."""
+    return 1000 + rank
+
+
+def job_tokens_per_s(world, tokens_per_step, steps, ms_max):
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ clocks -------------
 REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -228,7 +238,7 @@ def run_ours(args):
     per_set = 4 * B * H * N * d * 2
     R = max(2, math.ceil(4 * L2_BYTES / per_set))
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
+    g.manual_seed(rank_seed(rank))
     sets = []
     for _ in range(R):
         q, k, v = (torch.randn((B, H, N, d), generator=g, device=dev) / math.sqrt(d) for _ in range(3))
@@ -275,7 +285,7 @@ def run_ours(args):
     gpu_launches = args.steps * kernels_per_step
     ms_step = ms / args.steps
     tokens_step = B * N
-    value = world * tokens_step * args.steps / (ms / 1e3)
+    value = job_tokens_per_s(world, tokens_step, args.steps, ms)
     alg_bytes = 8 * B * H * N * d
     alg_flops = 6 * B * H * N * d * d
     achieved = alg_bytes / (ms_step / 1e3) / 1e9
@@ -351,7 +361,7 @@ def e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, steps, world, pg):
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(pg, e0.elapsed_time(e1), dev)
     nbytes = B * H * N * d * 2
-    return {"value": world * B * N * steps / (ms / 1e3), "unit": "tokens/s",
+    return {"value": job_tokens_per_s(world, B * N, steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
             "ms_per_step": ms / steps, "steps": steps,
             "note": "pinned host buffers, stream-ordered copies and the C-ABI call, eager launches"}
