@@ -55,12 +55,76 @@ def parse():
 
 
 def peaks():
+    """(HBM copy GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p.get("bf16_tflops_sustained", 1364.1)), "measured"
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured")
     except Exception:
-        return FALLBACK_HBM_GBS, 1400.0, "fallback"
+        return FALLBACK_HBM_GBS, 1590.0, 1400.0, "fallback"
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ device timing ------
+SLEEP_CYCLES = 4_000_000  # ~2 ms at 1.9 GHz: covers the host's graph submission
+
+
+def graph_timed(stream, dev, step, steps, pg=None, sampler=None):
+    """Capture `steps` calls of step(i) in one CUDA graph and time one replay with CUDA events
+    on `stream`.  A short device-side sleep is queued before the start event, so that the
+    host's submission of the replay happens while the GPU is busy and stays out of the timed
+    window.  Returns (ms for the whole replay, ms of the same replay timed without the sleep)."""
+    import torch
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        graph.capture_begin()
+        for i in range(steps):
+            step(i)
+        graph.capture_end()
+        graph.replay()  # upload and one warm replay (untimed)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the same replay with the host submission inside the window (reported separately)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_submit = e0.elapsed_time(e1)
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(SLEEP_CYCLES)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    ms = e0.elapsed_time(e1)
+    del graph
+    return ms, ms_submit
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
 
 
 # ------------------------------------------------------------------ rank plumbing ------
@@ -218,9 +282,69 @@ def cpu_oracle_rate(seconds, B, H, N, d, seed=0):
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": min(threads, per), "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{passes} passes of {per} units (b, h) x N={N} tokens each of the "
                       f"B={B} batch, {dt:.1f} s wall, fp64 per-token loops, one unit per thread"}
+
+
+def cpu_config_rates(target_s=1.5):
+    """The oracle's rate on each of the layer's workloads, on a bounded sample: whole images
+    (all heads or channels of one batch entry), doubled until a sample takes `target_s`, then
+    scaled to tokens/s.  Plus one single-thread time of the fp32 14x14 layer."""
+    import oracle
+    from linear_attention_split_b200 import inputs
+    threads = oracle.default_threads()
+    res = {"cpu_model": cpu_model(), "threads": threads}
+
+    def run(kind, B, kw, call):
+        n = 1
+        while True:
+            inp = inputs.make(kind, seed=0, B=n, **kw)
+            t0 = time.perf_counter()
+            call(inp)
+            dt = time.perf_counter() - t0
+            if dt >= target_s or n >= B:
+                break
+            n = min(B, n * 2)
+        N = kw.get("N", kw.get("Hg", 1) * kw.get("Wg", 1))
+        return {"tokens_per_s": n * N / dt, "sample": f"{n} of B={B} images, {dt:.2f} s",
+                "est_full_config_s": dt * B / n}
+
+    lin = lambda i: oracle.linear_fullbatch(i["q"], i["k"], i["v"], i["w0"], threads=threads)
+    res["linear_f32_14x14"] = run("linear", 1, dict(H=1, N=196, d=64, dtype="f32"), lin)
+    inp = inputs.linear_inputs(1, 1, 196, 64, dtype="f32")
+    t0 = time.perf_counter()
+    oracle.linear_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], threads=1)
+    res["linear_f32_14x14"]["single_thread_s"] = time.perf_counter() - t0
+    res["linear_vits_bf16"] = run("linear", 64, dict(H=6, N=196, d=64, dtype="bf16"), lin)
+    res["linear_56x56_bf16"] = run("linear", 32, dict(H=1, N=3136, d=64, dtype="bf16"), lin)
+    res["dwconv_56x56_bf16"] = run("dwconv", 32, dict(Hg=56, Wg=56, C=64, dtype="bf16"),
+                                   lambda i: oracle.dwconv_fullbatch(i["q"], i["k"], i["v"], i["w0"],
+                                                                     threads=threads))
+    res["mlp_64x64_bf16"] = run("mlp", 16, dict(H=12, N=4096, d=64, dtype="bf16"),
+                                lambda i: oracle.mlp_fullbatch(i["q"], i["k"], i["v"], i["w1"], i["w2"],
+                                                               threads=threads))
+    res["chunked_80x80_bf16"] = run("chunked", 8, dict(H=3, N=6400, d=64, dtype="bf16"),
+                                    lambda i: oracle.linear_chunked(i["q"], i["k"], i["v"], i["w0"], 64,
+                                                                    threads=threads))
+    return res
+
+
+def reference_sample(B, N, threads, unit_s, budget):
+    """Per-step sample of the reference arm: (units, tokens per unit, threads used).
+    Whole units (b, h) in passes of min(B, threads) parallel units while one pass fits the
+    per-step budget; otherwise min(B, threads) units, each cut to its first n tokens, n sized
+    so that the pass fits.  The oracle runs one unit per thread, so the threads used are
+    min(threads, units)."""
+    par = max(1, min(B, threads))
+    if budget >= unit_s:
+        units = max(1, min(B, int(budget / max(unit_s, 1e-9)) * par))
+        n = N
+    else:
+        units = par
+        n = max(16, min(N, int(N * budget / max(unit_s, 1e-9))))
+    return units, n, min(threads, units)
 
 
 # ------------------------------------------------------------------ our arm ------------
@@ -233,7 +357,7 @@ def run_ours(args):
         raise SystemExit("bench.py needs a CUDA device")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    hbm_peak, tf_peak, peak_src = peaks()
+    hbm_peak, tf_burst, tf_sust, peak_src = peaks()
     B, H, N, d, eta = WL["B"], WL["H"], WL["N"], WL["d"], WL["eta"]
     per_set = 4 * B * H * N * d * 2
     R = max(2, math.ceil(4 * L2_BYTES / per_set))
@@ -256,29 +380,10 @@ def run_ours(args):
             step(i)
     torch.cuda.synchronize(dev)
     assert ttt.device_error() == 0
-    # capture the K timed steps in one graph (launch overhead out of the measurement)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        graph.capture_begin()
-        for i in range(args.steps):
-            step(i)
-        graph.capture_end()
-    with torch.cuda.stream(stream):
-        graph.replay()  # graph upload and a warm replay (untimed)
-    torch.cuda.synchronize(dev)
+    # the K timed steps in one graph (launch overhead out of the measurement)
     launches0 = ttt.kernel_launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index)
-    barrier(pg, dev)
-    torch.cuda.synchronize(dev)
-    with sampler:
-        e0.record(stream)
-        with torch.cuda.stream(stream):
-            graph.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(pg, dev)
-    ms = e0.elapsed_time(e1)
+    ms, ms_submit = graph_timed(stream, dev, step, args.steps, pg=pg, sampler=sampler)
     ms = max_over_ranks(pg, ms, dev)
     assert ttt.device_error() == 0
     kernels_per_step = 1  # the tensor-core TTT-Linear path is a single kernel per call
@@ -292,7 +397,6 @@ def run_ours(args):
     traffic, sha = kernel_traffic(["linear_attention_split_b200/csrc/linear_tc5.cuh",
                                    "linear_attention_split_b200/csrc/common.cuh"],
                                   "linear_tc5_56x56.md")
-    del graph
 
     rec = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -304,7 +408,10 @@ def run_ours(args):
                    "parallelism": f"independent batches per rank (dp{world}), no collective",
                    "l2": f"{R} rotating input/output sets of {per_set / 1e6:.1f} MB "
                          f"({R * per_set / 1e6:.0f} MB > 4x L2)",
-                   "timing": "K steps in one CUDA graph, CUDA events on the launching stream"},
+                   "timing": "K steps in one CUDA graph, CUDA events on the launching stream; a "
+                             "device-side sleep before the start event keeps the host's graph "
+                             "submission out of the window",
+                   "graph_submit_ms_outside_window": max(0.0, ms_submit - ms)},
         "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
@@ -319,9 +426,10 @@ def run_ours(args):
 
     if not args.no_extras:
         rec["e2e"] = e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, min(args.steps, 200), world, pg)
-        rec["other_paths"] = other_paths(ttt, dev, stream, hbm_peak, tf_peak)
+        rec["other_paths"] = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust)
         if rank == 0 and world == 1:
             rec["cpu_baseline"] = cpu_oracle_rate(args.cpu_seconds, B, H, N, d)
+            rec["cpu_baseline"]["configs"] = cpu_config_rates()
         elif rank == 0:
             rec["cpu_baseline"] = None
     if rank == 0:
@@ -367,65 +475,76 @@ def e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, steps, world, pg):
             "note": "pinned host buffers, stream-ordered copies and the C-ABI call, eager launches"}
 
 
-def other_paths(ttt, dev, stream, hbm_peak, tf_peak, only=None, iters=None):
-    """Device time per call of the other paths at their workload shapes (informational).
-    `only` restricts the run to one path; `iters` overrides the timed call count."""
+def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=None):
+    """Device time per call of the other paths at their workload shapes.  Each path cycles
+    through rotating input/output sets whose total exceeds four times the L2 (so inputs come
+    from HBM), K calls in one CUDA graph, timed like the headline.  `only` restricts the run
+    to one path; `iters` overrides the timed call count."""
     import torch
     from linear_attention_split_b200 import inputs
     res = {}
 
-    def timed(fn, n):
-        n = iters if iters is not None else n
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                fn()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(n):
-                fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / n
+    def sets_for(per_set_bytes):
+        return max(2, math.ceil(4 * L2_BYTES / per_set_bytes))
+
+    def rotating(make, R):
+        out = []
+        for r in range(R):
+            inp = {k: v.to(dev) for k, v in make(r).items()}
+            inp["out"] = torch.empty_like(inp["q"])
+            out.append(inp)
+        return out
 
     def workspace(nbytes):
         return torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
 
+    def timed(fn, R, n):
+        n = iters if iters is not None else n
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                fn(i % R)
+        torch.cuda.synchronize(dev)
+        ms, _ = graph_timed(stream, dev, lambda i: fn(i % R), n)
+        return ms / n
+
     if only in (None, "dwconv"):  # 3x3 depthwise conv, B=32, 56x56, C=64
-        inp = {k: v.to(dev) for k, v in inputs.dwconv_inputs(32, 56, 56, 64).items()}
-        out = torch.empty_like(inp["q"])
-        ws = workspace(ttt.ttt_dwconv_fullbatch_workspace_bytes(32, 56, 56, 64, 1))
-        ms = timed(lambda: ttt.ttt_dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], out, None, 1.0,
-                                                    ws, stream), 20)
         nb = 8 * 32 * 3136 * 64
+        R = sets_for(nb)
+        S = rotating(lambda r: inputs.dwconv_inputs(32, 56, 56, 64, seed=100 + r), R)
+        ws = workspace(ttt.ttt_dwconv_fullbatch_workspace_bytes(32, 56, 56, 64, 1))
+        ms = timed(lambda i: ttt.ttt_dwconv_fullbatch(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"], S[i]["out"],
+                                                      None, 1.0, ws, stream), R, 200)
         res["dwconv_56x56_c64"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
                                    "hbm_gbs": nb / (ms / 1e3) / 1e9,
                                    "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / hbm_peak,
-                                   "note": "same inputs every call (51 MB, L2-resident), informational"}
-        del inp, out, ws
-    if only in (None, "mlp"):  # TTT-MLP, B=16, H=12, N=4096, d=64, h=256
-        inp = {k: v.to(dev) for k, v in inputs.mlp_inputs(16, 12, 4096, 64).items()}
-        out = torch.empty_like(inp["q"])
+                                   "l2": f"{R} rotating sets of {nb / 1e6:.1f} MB (> 4x L2)"}
+        del S, ws
+    if only in (None, "mlp"):  # TTT-MLP, B=16, H=12, N=4096, d=64, h=256 (403 MB per set)
+        R = 2
+        S = rotating(lambda r: inputs.mlp_inputs(16, 12, 4096, 64, seed=200 + r), R)
         ws = workspace(ttt.ttt_mlp_fullbatch_workspace_bytes(16, 12, 4096, 64, 256, 1))
-        ms = timed(lambda: ttt.ttt_mlp_fullbatch(inp["q"], inp["k"], inp["v"], inp["w1"], inp["w2"], out, None,
-                                                 None, 1.0, ws, stream), 5)
+        ms = timed(lambda i: ttt.ttt_mlp_fullbatch(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w1"], S[i]["w2"],
+                                                   S[i]["out"], None, None, 1.0, ws, stream), R, 10)
         fl = 14 * 16 * 12 * 4096 * 64 * 256
-        res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3),
-                                     "tflops": fl / (ms / 1e3) / 1e12,
-                                     "frac_of_tensor_peak": fl / (ms / 1e3) / 1e12 / tf_peak,
-                                     "peak": "sustained bf16 (MEASURED_PEAKS.json)"}
-        del inp, out, ws
+        tf = fl / (ms / 1e3) / 1e12
+        res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3), "tflops": tf,
+                                     "frac_of_tensor_peak": tf / tf_burst,
+                                     "frac_of_sustained_peak": tf / tf_sust,
+                                     "peak": "burst bf16 (MEASURED_PEAKS.json bf16_tflops): 10 calls, "
+                                             "a few ms in all"}
+        del S, ws
     if only in (None, "chunked"):  # chunked bidirectional, B=8, H=3, N=6400, d=64, chunk 64
-        inp = {k: v.to(dev) for k, v in inputs.chunked_inputs(8, 3, 6400, 64).items()}
-        out = torch.empty_like(inp["q"])
+        nb = 8 * 8 * 3 * 6400 * 64
+        R = sets_for(nb)
+        S = rotating(lambda r: inputs.chunked_inputs(8, 3, 6400, 64, seed=300 + r), R)
         ws = workspace(ttt.ttt_linear_chunked_bidir_workspace_bytes(8, 3, 6400, 64, 64, 1))
-        ms = timed(lambda: ttt.ttt_linear_chunked_bidir(inp["q"], inp["k"], inp["v"], inp["w0"], out, 64, 1.0,
-                                                        ws, stream), 5)
+        ms = timed(lambda i: ttt.ttt_linear_chunked_bidir(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"],
+                                                          S[i]["out"], 64, 1.0, ws, stream), R, 50)
         res["chunked_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
                                     "us_per_chunk_step": ms * 1e3 / 100,
-                                    "hbm_gbs_min_traffic": 8 * 8 * 3 * 6400 * 64 / (ms / 1e3) / 1e9}
-        del inp, out, ws
+                                    "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9,
+                                    "l2": f"{R} rotating sets of {nb / 1e6:.1f} MB (> 4x L2)"}
+        del S, ws
     assert ttt.device_error() == 0
     return res
 
@@ -436,9 +555,9 @@ def run_only(args):
     from linear_attention_split_b200 import ttt
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    hbm_peak, tf_peak, _ = peaks()
+    hbm_peak, tf_burst, tf_sust, _ = peaks()
     stream = torch.cuda.Stream(device=dev)
-    res = other_paths(ttt, dev, stream, hbm_peak, tf_peak, only=args.only, iters=args.steps)
+    res = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=args.only, iters=args.steps)
     print(json.dumps({"only": args.only, "steps": args.steps, "result": res}), flush=True)
 
 
@@ -455,16 +574,12 @@ def run_reference(args):
     threads = oracle.default_threads()
     inp = inputs.linear_inputs(B, H, N, d, dtype="bf16", seed=0)
     q, k, v, w0 = (oracle._f64(inp[x]) for x in ("q", "k", "v", "w0"))
-    # size each step so that warm-up + K steps stay within about two minutes: whole units
-    # (b, h) while one fits the per-step budget, else the first n tokens of one unit
+    # size each step so that warm-up + K steps stay within about two minutes
     t0 = time.perf_counter()
     oracle.linear_fullbatch(q[:1], k[:1], v[:1], w0, threads=1)
     unit_s = time.perf_counter() - t0
     budget = 120.0 / max(1, args.steps + args.warmup)
-    if budget >= unit_s:
-        units, n = max(1, min(B, threads, int(budget / max(unit_s, 1e-6) * min(threads, B)))), N
-    else:
-        units, n = 1, max(16, min(N, int(N * budget / max(unit_s, 1e-6))))
+    units, n, cores = reference_sample(B, N, threads, unit_s, budget)
     sl = slice(0, units)
     qs, ks, vs = (oracle._f64(x[sl, :, :n]) for x in (q, k, v))  # contiguous, copied once
     for _ in range(args.warmup):
@@ -475,15 +590,15 @@ def run_reference(args):
     dt = time.perf_counter() - t0
     value = units * n * args.steps / dt
     sample = (f"each step: {units} of the B={B} units (b, h), {n} of their N={N} tokens, d={d}, "
-              f"fp64 oracle, {threads} threads")
+              f"fp64 oracle, one unit per thread, {cores} threads")
     rec = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
            "config": {"workload": "TTT-Linear full-batch step, B=32 x 56x56 tokens (N=3136), 1 head, d=64, "
                                   "bf16 Q/K/V, fp32 W0, eta=1", "global_batch": B, "seq_len": N,
                       "parallelism": "host threads"},
-           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                            "sample": sample},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample, "cpu_model": cpu_model()},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(rec), flush=True)
 

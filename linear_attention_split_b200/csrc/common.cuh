@@ -12,8 +12,8 @@
 #include <stdint.h>
 
 #ifndef TTT_SPIN_LIMIT_CYCLES
-// Upper bound on any wait for data that another agent produces (TMA, another CTA): about
-// one second at the boost clock.  A wait that runs out records an error and moves on.
+// Default upper bound on any wait for data that another agent produces (TMA, the tensor
+// cores, another CTA): about one second at the boost clock.
 #define TTT_SPIN_LIMIT_CYCLES (2000000000LL)
 #endif
 
@@ -21,10 +21,25 @@
 #define TTT_DEVERR_TIMEOUT_TMA 0x1u      // a TMA transaction never completed
 #define TTT_DEVERR_TIMEOUT_PEER 0x2u     // a peer CTA never published its data
 #define TTT_DEVERR_BAD_LAUNCH 0x4u       // a kernel found its launch shape inconsistent
+#define TTT_DEVERR_TIMEOUT_ANY (TTT_DEVERR_TIMEOUT_TMA | TTT_DEVERR_TIMEOUT_PEER)
 
 __device__ unsigned int g_ttt_device_error;
+// Wait limit in SM clock cycles (host-settable for tests through ttt_debug_set_wait_limit).
+__device__ long long g_ttt_wait_limit = TTT_SPIN_LIMIT_CYCLES;
+// Test hook armed from the host (ttt_debug_arm_fault); 0 in normal operation.
+#define TTT_FAULT_SKIP_LOAD 0x1u         // the TTT-Linear producer leaves out its last K/V load
+__device__ unsigned int g_ttt_fault;
 
 __device__ __forceinline__ void ttt_raise(unsigned int bits) { atomicOr(&g_ttt_device_error, bits); }
+// True once any wait on this device has run out (until the host reads the error word): every
+// later wait then gives up at once, so one lost transfer costs one wait limit per kernel and
+// the kernel still reaches its normal teardown.
+__device__ __forceinline__ bool ttt_timed_out() {
+    return (*reinterpret_cast<volatile unsigned int*>(&g_ttt_device_error) & TTT_DEVERR_TIMEOUT_ANY) != 0;
+}
+__device__ __forceinline__ long long ttt_wait_limit() {
+    return *reinterpret_cast<volatile long long*>(&g_ttt_wait_limit);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,12 +90,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false (and raises `err`) if the phase never completes.
+// Bounded wait: returns false (and raises `err`) if the phase does not complete within the
+// wait limit, and at once if another wait on this device has already run out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int err) {
     if (mbar_try_wait(bar, parity)) return true;
+    const long long limit = ttt_wait_limit();
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > TTT_SPIN_LIMIT_CYCLES) {
+        if (ttt_timed_out()) return false;
+        if (clock64() - t0 > limit) {
             ttt_raise(err);
             return false;
         }

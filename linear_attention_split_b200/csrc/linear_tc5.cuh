@@ -93,6 +93,7 @@ __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.
 
 // Bounded wait with cluster-scope acquire (data written by peer CTAs with st.async).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int err) {
+    const long long limit = ttt_wait_limit();
     const long long t0 = clock64();
     for (;;) {
         uint32_t ok;
@@ -104,7 +105,8 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
             : "r"(smem_u32(bar)), "r"(parity)
             : "memory");
         if (ok) return true;
-        if (clock64() - t0 > TTT_SPIN_LIMIT_CYCLES) {
+        if (ttt_timed_out()) return false;
+        if (clock64() - t0 > limit) {
             ttt_raise(err);
             return false;
         }

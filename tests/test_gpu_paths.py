@@ -23,7 +23,8 @@ def check_dwconv(B, Hg, Wg, C, dtype, eta=1.0, seed=0):
     assert ttt.device_error() == 0
     ro, rw = oracle.dwconv_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"], eta=eta)
     dt = inp["q"].dtype
-    assert_close(out, ro, dt, f"dwconv O {B}x{Hg}x{Wg}x{C} {dtype}")
+    # heavy-tailed conv output: the bar is taken beyond the output's own bf16 rounding
+    assert_close(out, ro, dt, f"dwconv O {B}x{Hg}x{Wg}x{C} {dtype}", rounding_floor=True)
     assert_close(ws, rw, torch.float32 if dt == torch.float32 else dt, "dwconv w*")
 
 
@@ -52,26 +53,28 @@ def test_dwconv_f32():
 
 
 # ============================================================== TTT-MLP ===============
-def check_mlp(B, H, N, d, hidden, dtype, eta=1.0, seed=0, sample=None):
+def check_mlp(B, H, N, d, hidden, dtype, eta=1.0, seed=0):
     inp = inputs.mlp_inputs(B, H, N, d, hidden=hidden, dtype=dtype, seed=seed)
     g = cuda(inp)
     out, w1s, w2s = ttt.mlp_fullbatch(g["q"], g["k"], g["v"], g["w1"], g["w2"], eta=eta, with_w_star=True)
     assert ttt.device_error() == 0
     dt = inp["q"].dtype
     wdt = torch.float32 if dt == torch.float32 else dt
-    units = [(b, h) for b in range(B) for h in range(H)] if sample is None else sample
-    for b, h in units:
-        ro, r1, r2 = oracle.mlp_fullbatch(inp["q"][b:b + 1, h:h + 1], inp["k"][b:b + 1, h:h + 1],
-                                          inp["v"][b:b + 1, h:h + 1], inp["w1"][h:h + 1],
-                                          inp["w2"][h:h + 1], eta=eta)
-        assert_close(out[b:b + 1, h:h + 1], ro, dt, f"mlp O unit ({b},{h})")
-        assert_close(w1s[b:b + 1, h:h + 1], r1, wdt, f"mlp W1* unit ({b},{h})")
-        assert_close(w2s[b:b + 1, h:h + 1], r2, wdt, f"mlp W2* unit ({b},{h})")
+    # every unit at once (the oracle threads over units); each unit is also checked on its
+    # own so that a slip confined to one (b, h) cannot hide under the whole-tensor RMS
+    ro, r1, r2 = oracle.mlp_fullbatch(inp["q"], inp["k"], inp["v"], inp["w1"], inp["w2"], eta=eta)
+    assert_close(out, ro, dt, f"mlp O B={B} H={H} N={N}")
+    assert_close(w1s, r1, wdt, "mlp W1*")
+    assert_close(w2s, r2, wdt, "mlp W2*")
+    for b in range(B):
+        for h in range(H):
+            assert_close(out[b:b + 1, h:h + 1], ro[b:b + 1, h:h + 1], dt, f"mlp O unit ({b},{h})")
+    return out, w1s, w2s
 
 
-def test_mlp_64x64_bf16_sampled():
-    """Full shape B=16, 12 heads, N=4096, d=64, hidden 256, compared on sampled units."""
-    check_mlp(16, 12, 4096, 64, 256, "bf16", sample=[(0, 0), (3, 7), (15, 11), (9, 4)])
+def test_mlp_64x64_bf16_full():
+    """Full shape B=16, 12 heads, N=4096, d=64, hidden 256: all 192 units against the oracle."""
+    check_mlp(16, 12, 4096, 64, 256, "bf16")
 
 
 @pytest.mark.parametrize("N", [1, 100, 300, 1000])
@@ -126,3 +129,28 @@ def test_chunked_full_chunk_is_twice_fullbatch():
     out = ttt.linear_chunked_bidir(g["q"], g["k"], g["v"], g["w0"], 512)
     ref, _ = oracle.linear_fullbatch(inp["q"], inp["k"], inp["v"], inp["w0"])
     assert_close(out, 2 * ref, torch.bfloat16, "chunk = N")
+
+
+# ============================================================== determinism ===========
+def test_dwconv_deterministic_full_shape():
+    """Fixed-order reductions: two calls give bit-identical O and w* (B=32, 56x56, C=64)."""
+    g = cuda(inputs.dwconv_inputs(32, 56, 56, 64, dtype="bf16", seed=4))
+    o1, w1 = ttt.dwconv_fullbatch(g["q"], g["k"], g["v"], g["w0"], with_w_star=True)
+    o2, w2 = ttt.dwconv_fullbatch(g["q"], g["k"], g["v"], g["w0"], with_w_star=True)
+    assert torch.equal(o1, o2) and torch.equal(w1, w2)
+
+
+def test_mlp_deterministic_full_shape():
+    """Split-order partial sums: two calls give bit-identical O, W1*, W2* (B=16, H=12, N=4096)."""
+    g = cuda(inputs.mlp_inputs(16, 12, 4096, 64, dtype="bf16", seed=4))
+    r1 = ttt.mlp_fullbatch(g["q"], g["k"], g["v"], g["w1"], g["w2"], with_w_star=True)
+    r2 = ttt.mlp_fullbatch(g["q"], g["k"], g["v"], g["w1"], g["w2"], with_w_star=True)
+    assert all(torch.equal(a, b) for a, b in zip(r1, r2))
+
+
+def test_chunked_deterministic_full_shape():
+    """Parked partials combined in a fixed order: two calls give bit-identical O (80x80)."""
+    g = cuda(inputs.chunked_inputs(8, 3, 6400, 64, dtype="bf16", seed=4))
+    o1 = ttt.linear_chunked_bidir(g["q"], g["k"], g["v"], g["w0"], 64)
+    o2 = ttt.linear_chunked_bidir(g["q"], g["k"], g["v"], g["w0"], 64)
+    assert torch.equal(o1, o2)

@@ -234,6 +234,16 @@ def test_mlp_golden(golden_dir):
     np.testing.assert_allclose(out[0, 0], g["out"], rtol=rt)
 
 
+def test_mlp_golden_regenerates(golden_dir):
+    """The MLP fixture is reproduced bit for bit by its committed calculator program
+    (Python math only, nothing from the oracle)."""
+    import subprocess
+    import sys
+    script = os.path.join(golden_dir, "make_mlp_d1_h2.py")
+    r = subprocess.run([sys.executable, script, "--check"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def mlp_torch_loss(k, v, W1, W2):
     a = F.gelu(torch.tensor(k) @ W1, approximate="tanh")
     return 0.5 * ((a @ W2 - torch.tensor(v)) ** 2).sum(dim=1).mean()

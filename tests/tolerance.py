@@ -2,14 +2,15 @@
 
 fp32 inputs : max_i |o_i - r_i| / max(|r_i|, rms(r))   <= 1e-4  (max relative error with an RMS floor
               so that elements near zero do not dominate)
-bf16 inputs : max_i (|o_i - r_i| - u_i)+ / rms(r)       <= 2e-2  (fp32 accumulation on the GPU)
+bf16 inputs : max_i |o_i - r_i| / rms(r)                <= 2e-2  (fp32 accumulation on the GPU)
 r is the fp64 oracle result on the identical stored inputs.
 
-u_i is half a bf16 ulp at max(|o_i|, |r_i|) when the output itself is stored in bf16, and 0
-for fp32 outputs (W*, or fp32 layers).  Reading: the 2e-2 bar is on the arithmetic; a bf16
-output cannot be closer to the exact value than its own rounding, and for heavy-tailed
-outputs that rounding alone exceeds 2e-2 of the RMS (the 3x3 conv layer at 56x56, C = 64:
-max|o|/rms = 11.7, rounding floor 2.46e-2).  `raw_err` is reported beside it.
+The bf16 bar is applied to the raw difference.  One documented exception takes
+`rounding_floor=True`: the 3x3 conv layer at 56x56, C = 64, whose output is heavy-tailed
+(max|o|/rms = 11.7), so that the exact result rounded to bf16 is already 2.46e-2 of the RMS
+away from the exact value.  There, and only there, half a bf16 ulp at max(|o_i|, |r_i|) is
+taken off each difference before the bar (the bar then measures the arithmetic beyond the
+output's own rounding).  Both numbers are returned and printed.
 """
 import numpy as np
 import torch
@@ -29,28 +30,29 @@ def half_ulp_bf16(x):
     return np.where(a > 0, np.exp2(e - 8), 0.0)
 
 
-def err(gpu, ref, dtype, stored_bf16=None):
+def err(gpu, ref, dtype, rounding_floor=False):
+    """Returns (metric, raw): `metric` is what the bar applies to, `raw` = max|diff| / rms."""
     g = _np(gpu)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
     assert np.all(np.isfinite(g)), "non-finite GPU output"
-    if stored_bf16 is None:
-        stored_bf16 = hasattr(gpu, "dtype") and gpu.dtype == torch.bfloat16
+    stored_bf16 = hasattr(gpu, "dtype") and gpu.dtype == torch.bfloat16
     rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
     diff = np.abs(g - r)
-    raw = float(np.max(diff)) / rms if rms > 0 else float(np.max(diff, initial=0.0))
+    raw = float(np.max(diff, initial=0.0)) / rms if rms > 0 else float(np.max(diff, initial=0.0))
     if dtype == torch.float32:
         if rms == 0.0:
             return float(np.max(diff, initial=0.0)), raw
-        return float(np.max(diff / np.maximum(np.abs(r), rms))), raw
-    if stored_bf16:
+        return float(np.max(diff / np.maximum(np.abs(r), rms), initial=0.0)), raw
+    if rounding_floor and stored_bf16:
         diff = np.maximum(diff - half_ulp_bf16(np.maximum(np.abs(g), np.abs(r))), 0.0)
     if rms == 0.0:
         return float(np.max(diff, initial=0.0)), raw
-    return float(np.max(diff)) / rms, raw
+    return float(np.max(diff, initial=0.0)) / rms, raw
 
 
-def assert_close(gpu, ref, dtype, what=""):
-    e, raw = err(gpu, ref, dtype)
+def assert_close(gpu, ref, dtype, what="", rounding_floor=False):
+    e, raw = err(gpu, ref, dtype, rounding_floor=rounding_floor)
+    print(f"{what}: metric {e:.3e} raw max|diff|/rms {raw:.3e}")
     assert e <= TOL[dtype], f"{what}: error {e:.3e} > {TOL[dtype]:.0e} (raw max|diff|/rms {raw:.3e})"
     return e
