@@ -45,6 +45,14 @@ def lib():
         _lib.ttt_oracle_mlp_fullbatch.argtypes = [p, p, p, p, p, p, p, p, i, i, i, i, i, d, i]
         _lib.ttt_oracle_linear_chunked.restype = i
         _lib.ttt_oracle_linear_chunked.argtypes = [p, p, p, p, p, i, i, i, i, i, d, i, i]
+        _lib.ttt_oracle_linear_fullbatch_bwd.restype = i
+        _lib.ttt_oracle_linear_fullbatch_bwd.argtypes = [p, p, p, p, p, p, p, p, p, i, i, i, i, d, i]
+        _lib.ttt_oracle_linear_minibatch.restype = i
+        _lib.ttt_oracle_linear_minibatch.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, d, i]
+        _lib.ttt_oracle_dwconv_prep.restype = None
+        _lib.ttt_oracle_dwconv_prep.argtypes = [p, p, p, i, i, i, i, i]
+        _lib.ttt_oracle_linear_chunked_prep.restype = i
+        _lib.ttt_oracle_linear_chunked_prep.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, d, i, i]
     return _lib
 
 
@@ -171,6 +179,63 @@ def linear_chunked(q, k, v, w0, chunk, eta=1.0, direction=0, threads=None) -> np
     rc = lib().ttt_oracle_linear_chunked(_p(q), _p(k), _p(v), _p(w0), _p(out), B, H, N, d,
                                          int(chunk), float(eta), int(direction),
                                          threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return out
+
+
+# ---------------------------------------------------------------- backward --------------
+def linear_fullbatch_bwd(q, k, v, w0, dout, eta=1.0, threads=None):
+    """Gradients of the full-batch TTT-Linear layer for the upstream gradient `dout`:
+    q,k,v,dout [B,H,N,d]; w0 [H,d,d] -> (dq, dk, dv [B,H,N,d], dw0 [H,d,d] summed over B)."""
+    q, k, v, w0, g = _f64(q), _f64(k), _f64(v), _f64(w0), _f64(dout)
+    B, H, N, d = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    dw0 = np.empty((H, d, d))
+    rc = lib().ttt_oracle_linear_fullbatch_bwd(_p(q), _p(k), _p(v), _p(w0), _p(g), _p(dq), _p(dk),
+                                               _p(dv), _p(dw0), B, H, N, d, float(eta),
+                                               threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return dq, dk, dv, dw0
+
+
+# ---------------------------------------------------------------- mini-batch / epochs ---
+def linear_minibatch(q, k, v, w0, chunk, epochs=1, eta=1.0, threads=None):
+    """E epochs of mini-batch inner training in raster order, then out = Q W_final.
+    -> (out [B,H,N,d], w_final [B,H,d,d])."""
+    q, k, v, w0 = _f64(q), _f64(k), _f64(v), _f64(w0)
+    B, H, N, d = q.shape
+    out = np.empty_like(q)
+    wf = np.empty((B, H, d, d))
+    rc = lib().ttt_oracle_linear_minibatch(_p(q), _p(k), _p(v), _p(w0), _p(out), _p(wf), B, H, N, d,
+                                           int(chunk), int(epochs), float(eta),
+                                           threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return out, wf
+
+
+# ---------------------------------------------------------------- conv preprocessing ----
+def dwconv_prep(x, w, Hg, Wg):
+    """3x3 depthwise conv (zero padding) of x [B,H,Hg*Wg,d] with taps w [H,d,3,3]."""
+    x, w = _f64(x), _f64(w)
+    B, H, N, d = x.shape
+    assert N == Hg * Wg
+    out = np.empty_like(x)
+    lib().ttt_oracle_dwconv_prep(_p(x), _p(w), _p(out), B, H, Hg, Wg, d)
+    return out
+
+
+def linear_chunked_prep(q, k, v, w0, wk, wv, Hg, Wg, chunk, eta=1.0, direction=0, threads=None):
+    """Chunked scan on (Q, conv(K; wk), conv(V; wv)) over the Hg x Wg grid."""
+    q, k, v, w0, wk, wv = _f64(q), _f64(k), _f64(v), _f64(w0), _f64(wk), _f64(wv)
+    B, H, N, d = q.shape
+    assert N == Hg * Wg
+    out = np.empty_like(q)
+    rc = lib().ttt_oracle_linear_chunked_prep(_p(q), _p(k), _p(v), _p(w0), _p(wk), _p(wv), _p(out),
+                                              B, H, Hg, Wg, d, int(chunk), float(eta), int(direction),
+                                              threads or default_threads())
     if rc != 0:
         raise ValueError("oracle: bad arguments")
     return out

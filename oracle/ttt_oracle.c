@@ -485,3 +485,249 @@ int ttt_oracle_linear_chunked(const double* q, const double* k, const double* v,
     run_units((long)B * H, threads, chunked_unit, &c);
     return 0;
 }
+
+/* ==================================================================================== */
+/* Backward of TTT-Linear full batch (outer training through the inner step).          */
+/* Forward, per unit:  r_i = k_i W0 - v_i,  gW = (1/N) sum_i k_i^T r_i,                  */
+/*                     W* = W0 - eta gW,   o_j = q_j W*.                                 */
+/* Given the upstream gradient g_j = dL/do_j, the chain rule taken step by step back     */
+/* through those four lines (written out by hand, as the ViT^3 blog notes the official   */
+/* code does for the inner step, "从官方代码看…", third point):                            */
+/*   dW*    = sum_j q_j^T g_j            dq_j = g_j W*^T                                 */
+/*   dgW    = -eta dW*                   dW0 += dW*            (W* = W0 - eta gW)        */
+/*   dr_i   = (1/N) k_i dgW              dk_i += (1/N) r_i dgW^T   (gW = mean k^T r)     */
+/*   dk_i  += dr_i W0^T                  dv_i  = -dr_i          dW0 += k_i^T dr_i        */
+/* W0 is shared by the batch entries of a head, so dW0[h] = sum over b (b ascending).    */
+/* ==================================================================================== */
+
+typedef struct {
+    const double *q, *k, *v, *w0, *dout;
+    double *dq, *dk, *dv, *dw0_unit;
+    int H, N, d;
+    double eta;
+} linear_bwd_ctx;
+
+static void linear_bwd_unit(const void* vctx, long u) {
+    const linear_bwd_ctx* c = (const linear_bwd_ctx*)vctx;
+    const int d = c->d, N = c->N;
+    const long h = u % c->H;
+    const long tok = (long)N * d;
+    const long dd = (long)d * d;
+    const double* w0 = c->w0 + h * dd;
+    const double *q = c->q + u * tok, *k = c->k + u * tok, *v = c->v + u * tok;
+    const double* g = c->dout + u * tok;
+    double *dq = c->dq + u * tok, *dk = c->dk + u * tok, *dv = c->dv + u * tok;
+    double* dw0 = c->dw0_unit + u * dd;
+    double* gw = (double*)malloc(sizeof(double) * (size_t)dd);
+    double* ws = (double*)malloc(sizeof(double) * (size_t)dd);
+    double* dws = (double*)calloc((size_t)dd, sizeof(double));
+    double* dgw = (double*)malloc(sizeof(double) * (size_t)dd);
+    double* r = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dr = (double*)malloc(sizeof(double) * (size_t)d);
+    /* forward: gW and W* */
+    ttt_oracle_linear_grad(k, v, w0, N, d, gw);
+    for (long e = 0; e < dd; ++e) ws[e] = w0[e] - c->eta * gw[e];
+    /* o_j = q_j W*:  dW* = sum_j q_j^T g_j,  dq_j = g_j W*^T */
+    for (int t = 0; t < N; ++t) {
+        const double* qt = q + (long)t * d;
+        const double* gt = g + (long)t * d;
+        for (int a = 0; a < d; ++a)
+            for (int b = 0; b < d; ++b) dws[(long)a * d + b] += qt[a] * gt[b];
+        for (int a = 0; a < d; ++a) {
+            double s = 0.0;
+            for (int b = 0; b < d; ++b) s += gt[b] * ws[(long)a * d + b];
+            dq[(long)t * d + a] = s;
+        }
+    }
+    /* W* = W0 - eta gW */
+    for (long e = 0; e < dd; ++e) {
+        dgw[e] = -c->eta * dws[e];
+        dw0[e] = dws[e];
+    }
+    /* gW = (1/N) sum_i k_i^T r_i with r_i = k_i W0 - v_i, token by token */
+    for (int t = 0; t < N; ++t) {
+        const double* kt = k + (long)t * d;
+        const double* vt = v + (long)t * d;
+        for (int j = 0; j < d; ++j) {
+            double f = 0.0;
+            for (int m = 0; m < d; ++m) f += kt[m] * w0[(long)m * d + j];
+            r[j] = f - vt[j];
+        }
+        for (int b = 0; b < d; ++b) { /* dr_i = (1/N) k_i dgW */
+            double s = 0.0;
+            for (int a = 0; a < d; ++a) s += kt[a] * dgw[(long)a * d + b];
+            dr[b] = s / (double)N;
+        }
+        for (int a = 0; a < d; ++a) {
+            double s1 = 0.0, s2 = 0.0;
+            for (int b = 0; b < d; ++b) {
+                s1 += dgw[(long)a * d + b] * r[b];   /* (1/N) (r_i dgW^T)_a */
+                s2 += dr[b] * w0[(long)a * d + b];   /* (dr_i W0^T)_a      */
+            }
+            dk[(long)t * d + a] = s1 / (double)N + s2;
+        }
+        for (int b = 0; b < d; ++b) dv[(long)t * d + b] = -dr[b];
+        for (int a = 0; a < d; ++a)
+            for (int b = 0; b < d; ++b) dw0[(long)a * d + b] += kt[a] * dr[b];
+    }
+    free(gw);
+    free(ws);
+    free(dws);
+    free(dgw);
+    free(r);
+    free(dr);
+}
+
+int ttt_oracle_linear_fullbatch_bwd(const double* q, const double* k, const double* v,
+                                    const double* w0, const double* dout, double* dq,
+                                    double* dk, double* dv, double* dw0, int B, int H, int N,
+                                    int d, double eta, int threads) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 1;
+    const long dd = (long)d * d;
+    double* per_unit = (double*)malloc(sizeof(double) * (size_t)B * H * dd);
+    if (!per_unit) return 1;
+    linear_bwd_ctx c = {q, k, v, w0, dout, dq, dk, dv, per_unit, H, N, d, eta};
+    run_units((long)B * H, threads, linear_bwd_unit, &c);
+    for (int h = 0; h < H; ++h)
+        for (long e = 0; e < dd; ++e) {
+            double s = 0.0;
+            for (int b = 0; b < B; ++b) s += per_unit[((long)b * H + h) * dd + e];
+            dw0[h * dd + e] = s;
+        }
+    free(per_unit);
+    return 0;
+}
+
+/* ==================================================================================== */
+/* Mini-batch / multi-epoch inner training, then the trained model applied to Q.        */
+/* The inner-training options the ViT^3 blog's design study varies ("inner training 怎么 */
+/* 配": full batch or mini-batch, how many epochs): E epochs over the tokens in raster     */
+/* order, each epoch a sequence of mini-batches of b consecutive tokens,                 */
+/*     W <- W - (eta / b) sum_{t in chunk} k_t^T (k_t W - v_t)                            */
+/* (the online update rule of the Vision-TTT gist, item 1, per mini-batch as in item 3), */
+/* then o_t = q_t W_final for every token.  b = N and E = 1 is the full-batch step.      */
+/* ==================================================================================== */
+
+typedef struct {
+    const double *q, *k, *v, *w0;
+    double *out, *w_final;
+    int H, N, d, b, epochs;
+    double eta;
+} minibatch_ctx;
+
+static void minibatch_unit(const void* vctx, long u) {
+    const minibatch_ctx* c = (const minibatch_ctx*)vctx;
+    const int d = c->d, N = c->N, b = c->b;
+    const long h = u % c->H;
+    const long tok = (long)N * d;
+    const long dd = (long)d * d;
+    const double *k = c->k + u * tok, *v = c->v + u * tok;
+    double* w = (double*)malloc(sizeof(double) * (size_t)dd);
+    double* gc = (double*)malloc(sizeof(double) * (size_t)dd);
+    double* r = (double*)malloc(sizeof(double) * (size_t)d);
+    memcpy(w, c->w0 + h * dd, sizeof(double) * (size_t)dd);
+    for (int e = 0; e < c->epochs; ++e)
+        for (int c0 = 0; c0 < N; c0 += b) {
+            memset(gc, 0, sizeof(double) * (size_t)dd);
+            for (int t = c0; t < c0 + b; ++t) {
+                const double* kt = k + (long)t * d;
+                const double* vt = v + (long)t * d;
+                for (int j = 0; j < d; ++j) {
+                    double f = 0.0;
+                    for (int m = 0; m < d; ++m) f += kt[m] * w[(long)m * d + j];
+                    r[j] = f - vt[j];
+                }
+                for (int i = 0; i < d; ++i)
+                    for (int j = 0; j < d; ++j) gc[(long)i * d + j] += kt[i] * r[j];
+            }
+            for (long x = 0; x < dd; ++x) w[x] -= (c->eta / (double)b) * gc[x];
+        }
+    linear_apply(c->q + u * tok, w, N, d, c->out + u * tok);
+    if (c->w_final) memcpy(c->w_final + u * dd, w, sizeof(double) * (size_t)dd);
+    free(w);
+    free(gc);
+    free(r);
+}
+
+int ttt_oracle_linear_minibatch(const double* q, const double* k, const double* v,
+                                const double* w0, double* out, double* w_final, int B, int H,
+                                int N, int d, int chunk, int epochs, double eta, int threads) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || epochs <= 0) return 1;
+    if (N % chunk != 0) return 1;
+    minibatch_ctx c = {q, k, v, w0, out, w_final, H, N, d, chunk, epochs, eta};
+    run_units((long)B * H, threads, minibatch_unit, &c);
+    return 0;
+}
+
+/* ==================================================================================== */
+/* Conv2d preprocessing of the scan's dataset (Vision-TTT gist, item 2, "Conv2d Module":  */
+/* a depthwise convolution aggregates neighbouring tokens on the 2-D grid before the scan */
+/* starts; Vision-TTT review: "Conv2d-based dataset preprocessing").  Reading: the        */
+/* dataset is the (K, V) pairs; each of K and V goes through its own 3x3 depthwise conv   */
+/* on the Hg x Wg grid (one 3x3 filter per feature of each head, zero padding, no bias),  */
+/* then the chunked scan of the section above runs on (Q, K', V').                        */
+/* ==================================================================================== */
+
+void ttt_oracle_dwconv_prep(const double* x, const double* w, double* out, int B, int H,
+                            int Hg, int Wg, int d) {
+    const long N = (long)Hg * Wg;
+    for (long u = 0; u < (long)B * H; ++u) {
+        const long h = u % H;
+        const double* xu = x + u * N * d;
+        for (int y = 0; y < Hg; ++y)
+            for (int xx = 0; xx < Wg; ++xx)
+                for (int c = 0; c < d; ++c)
+                    out[u * N * d + ((long)y * Wg + xx) * d + c] =
+                        dwconv_at(xu, w + (h * d + c) * 9, Hg, Wg, d, y, xx, c);
+    }
+}
+
+typedef struct {
+    const double *q, *k, *v, *w0, *wk, *wv;
+    double* out;
+    int H, Hg, Wg, d, b, direction;
+    double eta;
+} chunked_prep_ctx;
+
+static void chunked_prep_unit(const void* vctx, long u) {
+    const chunked_prep_ctx* c = (const chunked_prep_ctx*)vctx;
+    const int d = c->d, N = c->Hg * c->Wg;
+    const long h = u % c->H;
+    const long tok = (long)N * d;
+    double* kp = (double*)malloc(sizeof(double) * (size_t)tok);
+    double* vp = (double*)malloc(sizeof(double) * (size_t)tok);
+    int* idx = (int*)calloc((size_t)N, sizeof(int));
+    /* K' and V' of this unit: one depthwise 3x3 filter per feature of head h */
+    for (int y = 0; y < c->Hg; ++y)
+        for (int x = 0; x < c->Wg; ++x)
+            for (int f = 0; f < d; ++f) {
+                const long at = ((long)y * c->Wg + x) * d + f;
+                kp[at] = dwconv_at(c->k + u * tok, c->wk + (h * d + f) * 9, c->Hg, c->Wg, d, y, x, f);
+                vp[at] = dwconv_at(c->v + u * tok, c->wv + (h * d + f) * 9, c->Hg, c->Wg, d, y, x, f);
+            }
+    double* o = c->out + u * tok;
+    memset(o, 0, sizeof(double) * (size_t)tok);
+    const double* w0 = c->w0 + h * (long)d * d;
+    if (c->direction >= 0) {
+        for (int t = 0; t < N; ++t) idx[t] = t;
+        chunked_scan(c->q + u * tok, kp, vp, w0, idx, N, d, c->b, c->eta, o);
+    }
+    if (c->direction <= 0) {
+        for (int t = 0; t < N; ++t) idx[t] = N - 1 - t;
+        chunked_scan(c->q + u * tok, kp, vp, w0, idx, N, d, c->b, c->eta, o);
+    }
+    free(kp);
+    free(vp);
+    free(idx);
+}
+
+int ttt_oracle_linear_chunked_prep(const double* q, const double* k, const double* v,
+                                   const double* w0, const double* wk, const double* wv,
+                                   double* out, int B, int H, int Hg, int Wg, int d, int chunk,
+                                   double eta, int direction, int threads) {
+    if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || d <= 0 || chunk <= 0) return 1;
+    if (direction < -1 || direction > 1) return 1;
+    chunked_prep_ctx c = {q, k, v, w0, wk, wv, out, H, Hg, Wg, d, chunk, direction, eta};
+    run_units((long)B * H, threads, chunked_prep_unit, &c);
+    return 0;
+}

@@ -44,6 +44,29 @@ int ttt_oracle_linear_chunked(const double* q, const double* k, const double* v,
                               const double* w0, double* out, int B, int H, int N, int d,
                               int chunk, double eta, int direction, int threads);
 
+/* backward of the full-batch TTT-Linear step: dout [B,H,N,d] -> dq, dk, dv [B,H,N,d],
+ * dw0 [H,d,d] (summed over the batch) */
+int ttt_oracle_linear_fullbatch_bwd(const double* q, const double* k, const double* v,
+                                    const double* w0, const double* dout, double* dq,
+                                    double* dk, double* dv, double* dw0, int B, int H, int N,
+                                    int d, double eta, int threads);
+
+/* E epochs of mini-batch inner training (chunks of `chunk` tokens, raster order), then
+ * out = Q W_final; w_final [B,H,d,d] or NULL */
+int ttt_oracle_linear_minibatch(const double* q, const double* k, const double* v,
+                                const double* w0, double* out, double* w_final, int B, int H,
+                                int N, int d, int chunk, int epochs, double eta, int threads);
+
+/* 3x3 depthwise conv of x [B,H,Hg*Wg,d] with taps w [H,d,3,3] (zero padding) */
+void ttt_oracle_dwconv_prep(const double* x, const double* w, double* out, int B, int H,
+                            int Hg, int Wg, int d);
+
+/* chunked scan on (Q, dwconv(K; wk), dwconv(V; wv)); wk, wv [H,d,3,3] */
+int ttt_oracle_linear_chunked_prep(const double* q, const double* k, const double* v,
+                                   const double* w0, const double* wk, const double* wv,
+                                   double* out, int B, int H, int Hg, int Wg, int d, int chunk,
+                                   double eta, int direction, int threads);
+
 #ifdef __cplusplus
 }
 #endif
