@@ -65,6 +65,19 @@ unsigned long long ttt_kernel_launch_count(void);
  * problem, TTT_ERR_TIMEOUT when a bounded wait ran out, TTT_ERR_CUDA on a CUDA failure. */
 int ttt_device_error(unsigned int* bits);
 
+/* Test support for the bounded waits (no counterpart on the pages).
+ * ttt_debug_set_wait_limit: the limit, in SM clock cycles, of every bounded wait in kernels
+ * launched afterwards on the current device; cycles <= 0 restores the default (about one
+ * second).  ttt_debug_arm_fault: arms (bits != 0) or clears (0) a simulated lost transfer on
+ * the current device: with TTT_FAULT_SKIP_LOAD set, the TTT-Linear tensor-core kernel (bf16,
+ * d = 64) leaves out the TMA load of each CTA's last K/V tile, so that the wait for it runs
+ * out and ttt_device_error() reports TTT_ERR_TIMEOUT.  Nothing faults: the kernel gives up the
+ * wait, computes on stale data and ends normally.  Both return TTT_OK or TTT_ERR_CUDA; each
+ * is a synchronous copy to the device, seen by kernels that start after it. */
+#define TTT_FAULT_SKIP_LOAD 0x1u
+int ttt_debug_set_wait_limit(long long cycles);
+int ttt_debug_arm_fault(unsigned int bits);
+
 /* --------------------------------------------------------------------------------------
  * TTT-Linear, full batch (F_W(x) = x W; TTT abstract of Sun et al.: "hidden state a linear
  * model").  Per unit u = b*H + h:
@@ -124,6 +137,54 @@ size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int 
 int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const float* w0,
                              void* out, int B, int H, int N, int d, int chunk, float eta,
                              int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * Chunked TTT-Linear scan in one direction or in both (Vision-TTT gist, "Technische
+ * samenvatting": item 1 the online update, item 2 the forward and backward scan, item 3 the
+ * mini-batches).  The recurrence is the one of ttt_linear_chunked_bidir above;
+ *   direction = +1: raster order only, O_c = Q_c W_c (the original one-way scan)
+ *   direction = -1: reverse raster order only
+ *   direction =  0: both, summed (identical to ttt_linear_chunked_bidir)
+ * Layouts and errors as for ttt_linear_chunked_bidir; direction outside {-1, 0, 1} is
+ * TTT_ERR_INVALID_ARG.  A one-way scan on the tensor-core path needs no workspace.
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_chunked_workspace_bytes(int B, int H, int N, int d, int chunk, int direction, int dtype);
+int ttt_linear_chunked(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H,
+                       int N, int d, int chunk, float eta, int direction, int dtype, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * Mini-batch / multi-epoch inner training of TTT-Linear, then the trained model applied to Q
+ * (the inner-training options that the ViT^3 blog's design study varies -- full batch or
+ * mini-batch, number of epochs -- with the per-mini-batch update of the Vision-TTT gist):
+ *     W <- W0[h];  repeat `epochs` times:  for each chunk c in raster order:
+ *                                            W <- W - (eta/chunk) K_c^T (K_c W - V_c)
+ *     O = Q W_final   (every token sees the final weights; nothing is output per chunk)
+ *   q, k, v, out : [B, H, N, d] dtype;  w0 : [H, d, d] fp32
+ *   w_final      : [B, H, d, d] fp32 output, or NULL
+ * chunk must divide N; epochs >= 1 (else TTT_ERR_INVALID_ARG).  chunk == N with one epoch is
+ * the full-batch step and runs ttt_linear_fullbatch.  The workspace is always needed.
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_minibatch_workspace_bytes(int B, int H, int N, int d, int chunk, int epochs, int dtype);
+int ttt_linear_minibatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_final,
+                         int B, int H, int N, int d, int chunk, int epochs, float eta, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
+ * Chunked scan on a Conv2d-preprocessed dataset (Vision-TTT gist, item 2 "Conv2d Module": a
+ * depthwise convolution aggregates neighbouring tokens of the 2-D grid before the scan;
+ * Vision-TTT review: "Conv2d-based dataset preprocessing").  This library's reading: each of
+ * K and V goes through its own 3x3 depthwise convolution on the Hg x Wg grid (one filter per
+ * feature of each head, zero padding, no bias), then ttt_linear_chunked runs on (Q, K', V').
+ *   q, k, v, out : [B, H, Hg*Wg, d] dtype (token index = row*Wg + col)
+ *   wk, wv       : [H, d, 3, 3] fp32 filters;  w0 : [H, d, d] fp32
+ * K' and V' are stored in the workspace in the input dtype; errors as for ttt_linear_chunked.
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_chunked_conv_workspace_bytes(int B, int H, int Hg, int Wg, int d, int chunk, int direction,
+                                               int dtype);
+int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const float* w0, const float* wk,
+                            const float* wv, void* out, int B, int H, int Hg, int Wg, int d, int chunk, float eta,
+                            int direction, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /* --------------------------------------------------------------------------------------
  * ttt_linear_chunked_bidir_noalloc -- the chunked bidirectional scan above, for callers that

@@ -25,6 +25,9 @@
 // and the combine of the two directions, which meet in the middle: at step s < nc/2 each
 // direction parks its fp32 partial output for its chunk in the workspace; at step s >= nc/2
 // it adds the partner's parked partial, rounds once to bf16 and stores O (deterministic).
+// A unidirectional scan (raster or reverse raster alone: the original, one-way TTT scan that
+// the Vision-TTT gist's bidirectional scan extends) runs one recurrence warp and one output
+// warp; the output warp rounds each chunk's O = Q_c W once and stores it, with nothing parked.
 #pragma once
 #include "common.cuh"
 
@@ -47,9 +50,11 @@ constexpr int PKB = CB * NCOL * 4;       // one chunk's partials for the CTA's c
 
 struct Params {
     const float* w0;    // [H][64][64]
-    float* park;        // workspace [U][N][64] fp32 (partial outputs)
+    float* park;        // workspace [U][N][64] fp32 (partial outputs; both directions only)
     __nv_bfloat16* out; // [U][N][64]
     int H, N, nc;       // nc = N / 64
+    int both;           // 1: both directions, summed; 0: direction `dir` alone
+    int dir;            // the direction of a one-way scan: 0 raster, 1 reverse raster
     float eta_over_b;
 };
 
@@ -76,6 +81,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto stage_ptr = [&](int dir, int s) { return ring + (dir * STAGES + s) * STAGE; };
     auto chunk_of = [&](int dir, int step) { return dir == 0 ? step : nc - 1 - step; };
     auto wfr_ptr = [&](int dir, int b) { return reinterpret_cast<uint4*>(wfr + (dir * WBUF + b) * WFR); };
+    auto active = [&](int dir) { return p.both || dir == p.dir; };
 
     if (threadIdx.x == 0) {
         for (int d = 0; d < 2; ++d) {
@@ -101,6 +107,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_prefetch_desc(&tm_v16);
             for (int step = 0; step < nc; ++step)
                 for (int dir = 0; dir < 2; ++dir) {
+                    if (!active(dir)) continue;
                     const int s = step % STAGES, use = step / STAGES;
                     if (use > 0) mbar_wait(&bars->empty[dir][s], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                     const int t0 = chunk_of(dir, step) * CB;
@@ -129,6 +136,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // = features 8 n..: wt[n] = {W[8n+2t][g], W[8n+2t+1][g], W[8n+2t][8+g], W[8n+2t+1][8+g]}
         // (column indices relative to this CTA's slice).
         const int dir = warp;
+        if (!active(dir)) return;
         float wt[8][4];
         {
             const float* W0 = p.w0 + (size_t)(u % p.H) * D * D + col0;
@@ -269,6 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // parks before all additions.  The partner's parked partials (64 tokens x 16 columns,
     // fp32) are fetched PF steps ahead by one TMA box each into a ring of PF + 1 slots.
     const int dir = warp - 2;
+    if (!active(dir)) return;
     uint8_t* pk = pkr + dir * (PF + 1) * PKB;
     const int a0 = (nc & 1) && dir == 0 ? nc / 2 + 1 : nc / 2;  // first step that adds
     auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st
@@ -330,6 +339,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         auto out_index = [&](int i, int j, int h) {
             return (tok0 + 16 * i + g + 8 * h) * D + col0 + 8 * j + 2 * t;
         };
+        if (!p.both) {  // one-way scan: this is the chunk's output
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<uint32_t*>(&p.out[out_index(i, j, h)]) = pack_bf16(o[i][j][2 * h], o[i][j][2 * h + 1]);
+            continue;
+        }
         if (step < a0) {  // first visit: park the fp32 partial
 #pragma unroll
             for (int i = 0; i < 4; ++i)

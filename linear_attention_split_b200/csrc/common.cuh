@@ -26,8 +26,8 @@
 __device__ unsigned int g_ttt_device_error;
 // Wait limit in SM clock cycles (host-settable for tests through ttt_debug_set_wait_limit).
 __device__ long long g_ttt_wait_limit = TTT_SPIN_LIMIT_CYCLES;
-// Test hook armed from the host (ttt_debug_arm_fault); 0 in normal operation.
-#define TTT_FAULT_SKIP_LOAD 0x1u         // the TTT-Linear producer leaves out its last K/V load
+// Test hook armed from the host (ttt_debug_arm_fault); 0 in normal operation.  Bit
+// TTT_FAULT_SKIP_LOAD (declared in ttt.h): the TTT-Linear producer leaves out its last K/V load.
 __device__ unsigned int g_ttt_fault;
 
 __device__ __forceinline__ void ttt_raise(unsigned int bits) { atomicOr(&g_ttt_device_error, bits); }
@@ -267,6 +267,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int mn_a, int mn_b) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)mn_a << 15) | ((uint32_t)mn_b << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// The same for fp16 A/B (both operands of one MMA share the type), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int mn_a, int mn_b) {
+    return (1u << 4) | ((uint32_t)mn_a << 15) | ((uint32_t)mn_b << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, int acc) {
     asm volatile(

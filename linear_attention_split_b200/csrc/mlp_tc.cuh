@@ -15,8 +15,11 @@
 //            K tile loads while the current tile's backward runs.  Each CTA writes its
 //            partial gradients (fp32) to the workspace.
 //   update : sums the partials of a unit in split order (deterministic) and forms W1*, W2*
-//            (fp32 outputs if requested, bf16 copies for the apply pass).
-//   apply  : per 128-token tile Z = Q W1*, A = gelu(Z), O = A W2*, stored as bf16 by TMA.
+//            (fp32 outputs if requested; for the apply pass W1* as bf16 hi + lo, W2* as fp16).
+//   apply  : per 128-token tile Z = Q W1*_hi + Q W1*_lo, A = gelu(Z) rounded to fp16,
+//            O = A W2* (fp16 x fp16, fp32 accumulate), stored as bf16 by TMA.  W1* is kept to
+//            2^-17 and A, W2* to 2^-11, so that O stays within a few tenths of a percent of the
+//            RMS of its exact value beyond the final bf16 rounding.
 // gelu uses the tanh form with the hardware tanh approximation (tanh.approx.f32).
 #pragma once
 #include "common.cuh"
@@ -426,8 +429,8 @@ struct UpdateParams {
     const float* part;          // [U][S][2][256][64]
     float* w1_star;             // [U][64][256] fp32 or nullptr
     float* w2_star;             // [U][256][64] fp32 or nullptr
-    __nv_bfloat16* w1b;         // [U][64][256] bf16
-    __nv_bfloat16* w2b;         // [U][256][64] bf16
+    __nv_bfloat16* w1b;         // [U][2][64][256] bf16: W1* hi, then lo = W1* - hi
+    __half* w2h;                // [U][256][64] fp16
     int H, S;
     float eta_over_n;
 };
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
         }
         const float w2 = p.w2[(size_t)hd * HID * D + h * D + tx] - p.eta_over_n * g2;  // W2*[h][d]
         if (p.w2_star) p.w2_star[(size_t)u * HID * D + h * D + tx] = w2;
-        p.w2b[(size_t)u * HID * D + h * D + tx] = __float2bfloat16_rn(w2);
+        p.w2h[(size_t)u * HID * D + h * D + tx] = __float2half_rn(w2);
         tile[rr][tx] = g1;  // gW1^T[h][d]
     }
     __syncthreads();
@@ -459,7 +462,9 @@ __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
         const size_t idx = (size_t)dd * HID + h0 + tx;
         const float w1 = p.w1[(size_t)hd * D * HID + idx] - p.eta_over_n * tile[tx][dd];
         if (p.w1_star) p.w1_star[(size_t)u * D * HID + idx] = w1;
-        p.w1b[(size_t)u * D * HID + idx] = __float2bfloat16_rn(w1);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
+        p.w1b[(size_t)u * 2 * D * HID + idx] = hi;
+        p.w1b[(size_t)u * 2 * D * HID + D * HID + idx] = __float2bfloat16_rn(w1 - __bfloat162float(hi));
     }
 }
 
@@ -475,15 +480,21 @@ struct ApplyBars {
 constexpr uint32_t COL_O = 256;  // apply: two 64-column O buffers after the two Z halves
 constexpr int NQB = 4;           // apply: Q tile buffers (O of a tile is staged over its Q tile)
 
+__device__ __forceinline__ uint32_t pack2_f16(uint64_t v) {
+    __half2 h = __floats2half2_rn(lo2(v), hi2(v));
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     apply_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                  const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
                  const ApplyParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* w1s = smem;
-    uint8_t* w2s = w1s + WBYTES;
-    uint8_t* at = w2s + WBYTES;
+    uint8_t* w1s = smem;                 // W1* hi (bf16)
+    uint8_t* w1l = w1s + WBYTES;         // W1* lo (bf16)
+    uint8_t* w2s = w1l + WBYTES;         // W2* (fp16)
+    uint8_t* at = w2s + WBYTES;          // A = gelu(Z) (fp16)
     uint8_t* qb = at + BIG;  // NQB x 16 KB: Q tiles, O staged in place
     ApplyBars* bars = reinterpret_cast<ApplyBars*>(qb + NQB * TILE);
 
@@ -517,7 +528,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_load_weights(w1s, w2s, &tm_w1, &tm_w2, u, &bars->wfull);  // this unit's W1*, W2*
+            // this unit's W1* hi and lo (rows 0-63 and 64-127 of its block) and W2*
+            mbar_expect_tx(&bars->wfull, 3 * WBYTES);
+#pragma unroll
+            for (int a = 0; a < HID / 64; ++a) {
+                tma_load_3d(w1s + a * 8192, &tm_w1, a * 64, 0, u, &bars->wfull);
+                tma_load_3d(w1l + a * 8192, &tm_w1, a * 64, D, u, &bars->wfull);
+            }
+            tma_load_3d(w2s, &tm_w2, 0, 0, u, &bars->wfull);
             for (int i = 0; i < ntiles; ++i) {
                 const int b = i % NQB;
                 if (i >= NQB) mbar_wait(&bars->qfree[b], (i / NQB - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
@@ -530,15 +548,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         // Z in two hidden halves (T0, T1) and O in two buffers: Z0 of tile i+1 is issued once
         // the epilogue has read Z0 of tile i, while it still works on Z1 and on O of tile i.
         if (lane == 0 && ntiles > 0) {
-            const uint32_t w1a = smem_u32(w1s), w2a = smem_u32(w2s), aa = smem_u32(at);
+            const uint32_t w1a = smem_u32(w1s), w1b = smem_u32(w1l), w2a = smem_u32(w2s), aa = smem_u32(at);
             const uint32_t IZ = tc::idesc_bf16(128, 128, 0, 1);
-            const uint32_t IO = tc::idesc_bf16(128, 64, 0, 1);
+            const uint32_t IO = tc::idesc_f16(128, 64, 0, 1);
             auto issue_z = [&](int i, int half) {
                 const uint32_t qa = smem_u32(qb + (i % NQB) * TILE);
                 tc::fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
                                  tc::smem_desc(w1a + half * 2 * 8192 + ks * 2048, 8192, 1024, 2), IZ, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_T + half * 128, tc::smem_desc(qa + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(w1b + half * 2 * 8192 + ks * 2048, 8192, 1024, 2), IZ, 1);
                 tc::commit(half ? &bars->z1full : &bars->z0full);
             };
             mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
@@ -612,7 +633,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int j = 0; j < 64; j += 8) {
                     uint32_t a[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) a[e] = pack2_bf16(gelu2(pk2(z[j + 2 * e], z[j + 2 * e + 1])));
+                    for (int e = 0; e < 4; ++e) a[e] = pack2_f16(gelu2(pk2(z[j + 2 * e], z[j + 2 * e + 1])));
                     *reinterpret_cast<uint4*>(at + big_off(r, c0 + j)) = make_uint4(a[0], a[1], a[2], a[3]);
                 }
                 fence_proxy_async_smem();

@@ -240,23 +240,24 @@ __global__ void __launch_bounds__(TPB) mlp_update_w2(const float* __restrict__ a
 // ------------------------------------------------------------------ chunked scan -----
 // One block per (unit, direction).  Shared memory: W [d][d], G [d][d], R [RB][d] (fp32).
 // Direction 0 visits chunks 0..nc-1, direction 1 visits them nc-1..0 (reverse raster);
-// the order of tokens inside a chunk does not change its sums.
+// the order of tokens inside a chunk does not change its sums.  The grid's y extent is the
+// number of directions run (1 or 2), the first of them is dir0; each writes its own partial.
 constexpr int CH_RB = 32;
 
 template <typename T>
 __global__ void __launch_bounds__(TPB) chunked_scan(const T* __restrict__ q, const T* __restrict__ k,
                                                     const T* __restrict__ v, const float* __restrict__ w0,
                                                     float* __restrict__ opart, int H, int N, int d, int chunk,
-                                                    float eta_over_b) {
+                                                    float eta_over_b, int dir0) {
     extern __shared__ float sm[];
     float* W = sm;
     float* G = W + d * d;
     float* R = G + d * d;
     const long long u = blockIdx.x;
-    const int dir = blockIdx.y;
+    const int dir = dir0 + (int)blockIdx.y;
     const int dd = d * d;
     const long long base = u * N * d;
-    float* op = opart + (long long)dir * gridDim.x * N * d + base;
+    float* op = opart + (long long)blockIdx.y * gridDim.x * N * d + base;
     for (int e = threadIdx.x; e < dd; e += TPB) W[e] = w0[(u % H) * dd + e];
     __syncthreads();
     const int nc = N / chunk;
@@ -299,10 +300,87 @@ __global__ void __launch_bounds__(TPB) chunked_scan(const T* __restrict__ q, con
 
 template <typename T>
 __global__ void __launch_bounds__(TPB) chunked_combine(const float* __restrict__ opart, T* __restrict__ out,
-                                                       long long total) {
+                                                       long long total, int nparts) {
     const long long e = (long long)blockIdx.x * TPB + threadIdx.x;
     if (e >= total) return;
-    out[e] = from_f<T>(opart[e] + opart[total + e]);
+    out[e] = from_f<T>(nparts == 2 ? opart[e] + opart[total + e] : opart[e]);
+}
+
+// ------------------------------------------------------------------ mini-batch training --
+// One block per unit: E epochs over the chunks in raster order, W <- W - (eta/b) K_c^T (K_c W
+// - V_c), nothing output per chunk; W_final (fp32) goes to wfin[u] (and w_out[u] if given).
+template <typename T>
+__global__ void __launch_bounds__(TPB) minibatch_train(const T* __restrict__ k, const T* __restrict__ v,
+                                                       const float* __restrict__ w0, float* __restrict__ wfin,
+                                                       float* __restrict__ w_out, int H, int N, int d, int chunk,
+                                                       int epochs, float eta_over_b) {
+    extern __shared__ float sm[];
+    float* W = sm;
+    float* G = W + d * d;
+    float* R = G + d * d;
+    const long long u = blockIdx.x;
+    const int dd = d * d;
+    const long long base = u * N * d;
+    for (int e = threadIdx.x; e < dd; e += TPB) W[e] = w0[(u % H) * dd + e];
+    __syncthreads();
+    const int nc = N / chunk;
+    for (int ep = 0; ep < epochs; ++ep)
+        for (int ci = 0; ci < nc; ++ci) {
+            const int c0 = ci * chunk;
+            for (int e = threadIdx.x; e < dd; e += TPB) G[e] = 0.f;
+            __syncthreads();
+            for (int s0 = 0; s0 < chunk; s0 += CH_RB) {
+                const int nr = min(CH_RB, chunk - s0);
+                for (int e = threadIdx.x; e < nr * d; e += TPB) {  // residuals with W before the update
+                    const int tt = e / d, j = e % d;
+                    const long long t = c0 + s0 + tt;
+                    float f = 0.f;
+                    for (int m = 0; m < d; ++m) f = fmaf(to_f(k[base + t * d + m]), W[m * d + j], f);
+                    R[e] = f - to_f(v[base + t * d + j]);
+                }
+                __syncthreads();
+                for (int e = threadIdx.x; e < dd; e += TPB) {
+                    const int i = e / d, j = e % d;
+                    float g = G[e];
+                    for (int tt = 0; tt < nr; ++tt) g = fmaf(to_f(k[base + (long long)(c0 + s0 + tt) * d + i]), R[tt * d + j], g);
+                    G[e] = g;
+                }
+                __syncthreads();
+            }
+            for (int e = threadIdx.x; e < dd; e += TPB) W[e] -= eta_over_b * G[e];
+            __syncthreads();
+        }
+    for (int e = threadIdx.x; e < dd; e += TPB) {
+        wfin[u * dd + e] = W[e];
+        if (w_out) w_out[u * dd + e] = W[e];
+    }
+}
+
+// ------------------------------------------------------------------ conv preprocessing --
+// x' = 3x3 depthwise conv of x over the Hg x Wg token grid of each unit (zero padding, no
+// bias): one filter per feature of each head, taps w [H][d][3][3]; x, y [U][Hg*Wg][d].
+template <typename T>
+__global__ void __launch_bounds__(TPB) dwconv_prep(const T* __restrict__ x, const float* __restrict__ w,
+                                                   T* __restrict__ y, int H, int Hg, int Wg, int d) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    const long long N = (long long)Hg * Wg;
+    if (e >= N * d) return;
+    const int f = (int)(e % d);
+    const long long t = e / d;
+    const int py = (int)(t / Wg), px = (int)(t % Wg);
+    const float* wf = w + ((u % H) * d + f) * 9;
+    const T* xu = x + u * N * d;
+    float acc = 0.f;
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            const int yy = py + a - 1, xx = px + b - 1;
+            if (yy >= 0 && yy < Hg && xx >= 0 && xx < Wg)
+                acc = fmaf(wf[a * 3 + b], to_f(xu[((long long)yy * Wg + xx) * d + f]), acc);
+        }
+    y[u * N * d + e] = from_f<T>(acc);
 }
 
 }  // namespace simt

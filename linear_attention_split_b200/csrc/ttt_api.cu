@@ -99,16 +99,16 @@ bool tmap_bf16_3d(CUtensorMap* m, const void* base, int d, int N, int U, int box
 }
 
 // ------------------------------------------------------------------ TTT-Linear --------
-// bf16 tensor [dim2][dim1][dim0] (dim0 fastest) viewed as 3-D, box {box0, box1, 1}
+// 16-bit tensor [dim2][dim1][dim0] (dim0 fastest) viewed as 3-D, box {box0, box1, 1}
 bool tmap_bf16_box(CUtensorMap* m, const void* base, int dim0, int dim1, int dim2, int box0, int box1,
-                   CUtensorMapSwizzle sw) {
+                   CUtensorMapSwizzle sw, CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
     cuuint64_t strides[2] = {(cuuint64_t)dim0 * 2, (cuuint64_t)dim1 * dim0 * 2};
     cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(m, type, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -424,8 +424,8 @@ size_t mlp_tc_ws(int B, int H, int N) {
     const int sms = current_device(&dev) == TTT_OK ? dev->sms : 148;
     const long long U = (long long)B * H;
     const int S = mlp_splits(U, N, sms);
-    return align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4) + 2 * align256((size_t)U * mlp::D * mlp::HID * 2) +
-           2 * align256((size_t)H * mlp::D * mlp::HID * 2);
+    return align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4) + align256((size_t)U * 2 * mlp::D * mlp::HID * 2) +
+           align256((size_t)U * mlp::D * mlp::HID * 2) + 2 * align256((size_t)H * mlp::D * mlp::HID * 2);
 }
 
 int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
@@ -438,9 +438,9 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     char* w = static_cast<char*>(ws);
     float* part = reinterpret_cast<float*>(w);
     w += align256((size_t)U * S * 2 * mlp::HID * mlp::D * 4);
-    __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(w);
-    w += align256((size_t)U * mlp::D * mlp::HID * 2);
-    __nv_bfloat16* w2b = reinterpret_cast<__nv_bfloat16*>(w);
+    __nv_bfloat16* w1b = reinterpret_cast<__nv_bfloat16*>(w);  // W1* hi and lo per unit
+    w += align256((size_t)U * 2 * mlp::D * mlp::HID * 2);
+    __half* w2h16 = reinterpret_cast<__half*>(w);               // W2* in fp16
     w += align256((size_t)U * mlp::D * mlp::HID * 2);
     __nv_bfloat16* w1h = reinterpret_cast<__nv_bfloat16*>(w);   // W1, W2 of every head in bf16
     w += align256((size_t)H * mlp::D * mlp::HID * 2);
@@ -452,12 +452,12 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
         !tmap_bf16_3d(&to, out, 64, N, U, 32, sw) ||
         !tmap_bf16_box(&tw1h, w1h, mlp::HID, mlp::D, H, 64, 64, sw) ||
         !tmap_bf16_box(&tw2h, w2h, mlp::D, mlp::HID, H, 64, mlp::HID, sw) ||
-        !tmap_bf16_box(&tw1s, w1b, mlp::HID, mlp::D, U, 64, 64, sw) ||
-        !tmap_bf16_box(&tw2s, w2b, mlp::D, mlp::HID, U, 64, mlp::HID, sw))
+        !tmap_bf16_box(&tw1s, w1b, mlp::HID, 2 * mlp::D, U, 64, 64, sw) ||
+        !tmap_bf16_box(&tw2s, w2h16, mlp::D, mlp::HID, U, 64, mlp::HID, sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return TTT_ERR_CUDA;
     const int smem_g = 2 * mlp::WBYTES + 2 * mlp::BIG + 2 * mlp::TILE + (int)sizeof(mlp::GradBars) + 1024;
-    const int smem_a = 2 * mlp::WBYTES + mlp::BIG + mlp::NQB * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
-    if (smem_g > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    const int smem_a = 3 * mlp::WBYTES + mlp::BIG + mlp::NQB * mlp::TILE + (int)sizeof(mlp::ApplyBars) + 1024;
+    if (smem_g > dev->smem_optin || smem_a > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(mlp::grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_g) != cudaSuccess ||
         cudaFuncSetAttribute(mlp::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
         return TTT_ERR_CUDA;
@@ -477,7 +477,7 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
     up.w1_star = w1_star;
     up.w2_star = w2_star;
     up.w1b = w1b;
-    up.w2b = w2b;
+    up.w2h = w2h16;
     up.H = H;
     up.S = S;
     up.eta_over_n = (float)((double)eta / (double)N);
@@ -490,15 +490,21 @@ int mlp_tc(const void* q, const void* k, const void* v, const float* w1, const f
 }
 
 // ------------------------------------------------------------------ chunked scan ------
-size_t chunked_ws(int B, int H, int N, int d) { return align256((size_t)2 * B * H * N * d * 4); }
+// direction: 0 both scans summed, +1 raster only, -1 reverse raster only
+int n_dirs(int direction) { return direction == 0 ? 2 : 1; }
+size_t chunked_ws(int B, int H, int N, int d, int direction) {
+    return align256((size_t)n_dirs(direction) * B * H * N * d * 4);
+}
 
 bool chunked_tc_ok(int B, int H, int d, int chunk, int dtype) {
     return dtype == TTT_BF16 && d == chk::D && chunk == chk::CB && (long long)B * H <= 65535;
 }
-size_t chunked_tc_ws(int B, int H, int N) { return align256((size_t)B * H * N * chk::D * 4); }
+size_t chunked_tc_ws(int B, int H, int N, int direction) {
+    return direction == 0 ? align256((size_t)B * H * N * chk::D * 4) : 0;  // parked partials
+}
 
 int chunked_tc(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
-               float eta, void* ws, cudaStream_t st) {
+               float eta, int direction, void* ws, cudaStream_t st) {
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     const int U = B * H;
@@ -509,6 +515,8 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
     p.H = H;
     p.N = N;
     p.nc = N / chk::CB;
+    p.both = direction == 0 ? 1 : 0;
+    p.dir = direction < 0 ? 1 : 0;
     p.eta_over_b = (float)((double)eta / (double)chk::CB);
     const int smem = 2 * chk::STAGES * chk::STAGE + 2 * chk::WBUF * chk::WFR + 2 * (chk::PF + 1) * chk::PKB +
                      (int)sizeof(chk::Bars) + 1024;
@@ -528,9 +536,11 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return TTT_ERR_CUDA;
-        // parked partials (fp32 [U][N][64]): box of 16 columns x 64 tokens, no swizzle
+        // parked partials (fp32 [U][N][64]): box of 16 columns x 64 tokens, no swizzle (a one-way
+        // scan parks nothing and never uses this map; it is encoded over `out` then)
         cuuint64_t pstrides[2] = {256, (cuuint64_t)N * 256};
-        if (fn(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws, dims, pstrides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        void* pbase = ws ? ws : out;
+        if (fn(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, pbase, dims, pstrides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return TTT_ERR_CUDA;
@@ -544,7 +554,7 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
 
 template <typename T>
 int chunked_simt(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
-                 int d, int chunk, float eta, void* ws, cudaStream_t st) {
+                 int d, int chunk, float eta, int direction, void* ws, cudaStream_t st) {
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     const long long U = (long long)B * H;
@@ -557,11 +567,11 @@ int chunked_simt(const void* q, const void* k, const void* v, const float* w0, v
         return TTT_ERR_CUDA;
     float* op = static_cast<float*>(ws);
     const float eta_over_b = (float)((double)eta / (double)chunk);
-    simt::chunked_scan<T><<<dim3((unsigned)U, 2), simt::TPB, smem, st>>>(
+    simt::chunked_scan<T><<<dim3((unsigned)U, n_dirs(direction)), simt::TPB, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), w0, op, H, N, d, chunk,
-        eta_over_b);
+        eta_over_b, direction < 0 ? 1 : 0);
     simt::chunked_combine<T><<<(unsigned)((total + simt::TPB - 1) / simt::TPB), simt::TPB, 0, st>>>(
-        op, static_cast<T*>(out), total);
+        op, static_cast<T*>(out), total, n_dirs(direction));
     return launched(2);
 }
 
@@ -617,6 +627,15 @@ int ttt_device_error(unsigned int* bits) {
     if (bits) *bits = v;
     if (v & (TTT_DEVERR_TIMEOUT_TMA | TTT_DEVERR_TIMEOUT_PEER)) return TTT_ERR_TIMEOUT;
     return v ? TTT_ERR_CUDA : TTT_OK;
+}
+
+int ttt_debug_set_wait_limit(long long cycles) {
+    const long long v = cycles > 0 ? cycles : (long long)TTT_SPIN_LIMIT_CYCLES;
+    return cudaMemcpyToSymbol(g_ttt_wait_limit, &v, sizeof(v)) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int ttt_debug_arm_fault(unsigned int bits) {
+    return cudaMemcpyToSymbol(g_ttt_fault, &bits, sizeof(bits)) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ TTT-Linear --------
@@ -694,26 +713,141 @@ int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* 
 }
 
 // ------------------------------------------------------------------ chunked scan ------
+size_t ttt_linear_chunked_workspace_bytes(int B, int H, int N, int d, int chunk, int direction, int dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || direction < -1 || direction > 1) return 0;
+    if (chunked_tc_ok(B, H, d, chunk, dtype)) return chunked_tc_ws(B, H, N, direction);
+    return chunked_ws(B, H, N, d, direction);
+}
+
+int ttt_linear_chunked(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H,
+                       int N, int d, int chunk, float eta, int direction, int dtype, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w0 || !aligned16(w0)) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0) return TTT_ERR_INVALID_ARG;
+    if (direction < -1 || direction > 1) return TTT_ERR_INVALID_ARG;
+    if (d > 128) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, direction, dtype);
+    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (chunked_tc_ok(B, H, d, chunk, dtype))
+        return chunked_tc(q, k, v, w0, out, B, H, N, eta, direction, need ? workspace : nullptr, st);
+    if (dtype == TTT_BF16)
+        return chunked_simt<__nv_bfloat16>(q, k, v, w0, out, B, H, N, d, chunk, eta, direction, workspace, st);
+    return chunked_simt<float>(q, k, v, w0, out, B, H, N, d, chunk, eta, direction, workspace, st);
+}
+
 size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int chunk, int dtype) {
-    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-    if (chunked_tc_ok(B, H, d, chunk, dtype)) return chunked_tc_ws(B, H, N);
-    return chunked_ws(B, H, N, d);
+    return ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, 0, dtype);
 }
 
 int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const float* w0, void* out, int B,
                              int H, int N, int d, int chunk, float eta, int dtype, void* workspace,
                              size_t workspace_bytes, void* stream) {
+    return ttt_linear_chunked(q, k, v, w0, out, B, H, N, d, chunk, eta, 0, dtype, workspace, workspace_bytes,
+                              stream);
+}
+
+// ------------------------------------------------------------------ mini-batch training --
+size_t ttt_linear_minibatch_workspace_bytes(int B, int H, int N, int d, int chunk, int epochs, int dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || epochs <= 0) return 0;
+    const size_t own = align256((size_t)B * H * d * d * 4);
+    if (chunk == N && epochs == 1) return std::max(own, ttt_linear_fullbatch_workspace_bytes(B, H, N, d, dtype));
+    return own;
+}
+
+int ttt_linear_minibatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_final,
+                         int B, int H, int N, int d, int chunk, int epochs, float eta, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
-    if (!w0 || !aligned16(w0)) return TTT_ERR_INVALID_ARG;
-    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0) return TTT_ERR_INVALID_ARG;
+    if (!w0 || !aligned16(w0) || (w_final && !aligned16(w_final))) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0 || epochs <= 0)
+        return TTT_ERR_INVALID_ARG;
     if (d > 128) return TTT_ERR_UNSUPPORTED;
-    const size_t need = ttt_linear_chunked_bidir_workspace_bytes(B, H, N, d, chunk, dtype);
-    if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    const size_t need = ttt_linear_minibatch_workspace_bytes(B, H, N, d, chunk, epochs, dtype);
+    if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    // one epoch over one chunk of all N tokens is the full-batch step
+    if (chunk == N && epochs == 1)
+        return ttt_linear_fullbatch(q, k, v, w0, out, w_final, B, H, N, d, eta, dtype, workspace, workspace_bytes,
+                                    stream);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (chunked_tc_ok(B, H, d, chunk, dtype)) return chunked_tc(q, k, v, w0, out, B, H, N, eta, workspace, st);
-    if (dtype == TTT_BF16)
-        return chunked_simt<__nv_bfloat16>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
-    return chunked_simt<float>(q, k, v, w0, out, B, H, N, d, chunk, eta, workspace, st);
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const long long U = (long long)B * H;
+    if (!grid_ok(U, (long long)N * d) || U > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+    const int smem = (2 * d * d + simt::CH_RB * d) * 4;
+    if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+    float* wfin = static_cast<float*>(workspace);
+    const float eta_over_b = (float)((double)eta / (double)chunk);
+    if (dtype == TTT_BF16) {
+        using T = __nv_bfloat16;
+        if (cudaFuncSetAttribute(simt::minibatch_train<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return TTT_ERR_CUDA;
+        simt::minibatch_train<T><<<(unsigned)U, simt::TPB, smem, st>>>(
+            static_cast<const T*>(k), static_cast<const T*>(v), w0, wfin, w_final, H, N, d, chunk, epochs, eta_over_b);
+        simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(static_cast<const T*>(q), wfin,
+                                                                                    static_cast<T*>(out), N, d);
+    } else {
+        using T = float;
+        if (cudaFuncSetAttribute(simt::minibatch_train<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return TTT_ERR_CUDA;
+        simt::minibatch_train<T><<<(unsigned)U, simt::TPB, smem, st>>>(
+            static_cast<const T*>(k), static_cast<const T*>(v), w0, wfin, w_final, H, N, d, chunk, epochs, eta_over_b);
+        simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(static_cast<const T*>(q), wfin,
+                                                                                    static_cast<T*>(out), N, d);
+    }
+    return launched(2);
+}
+
+// ------------------------------------------------------------------ conv-preprocessed scan
+size_t ttt_linear_chunked_conv_workspace_bytes(int B, int H, int Hg, int Wg, int d, int chunk, int direction,
+                                               int dtype) {
+    if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || d <= 0) return 0;
+    const long long N = (long long)Hg * Wg;
+    if (N > 0x7fffffffLL) return 0;
+    const size_t es = dtype == TTT_BF16 ? 2 : 4;
+    return 2 * align256((size_t)B * H * N * d * es) +
+           ttt_linear_chunked_workspace_bytes(B, H, (int)N, d, chunk, direction, dtype);
+}
+
+int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const float* w0, const float* wk,
+                            const float* wv, void* out, int B, int H, int Hg, int Wg, int d, int chunk, float eta,
+                            int direction, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
+    if (!w0 || !wk || !wv || !aligned16(w0) || !aligned16(wk) || !aligned16(wv)) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || d <= 0 || chunk <= 0) return TTT_ERR_INVALID_ARG;
+    const long long N = (long long)Hg * Wg;
+    if (N > 0x7fffffffLL || N % chunk != 0 || direction < -1 || direction > 1) return TTT_ERR_INVALID_ARG;
+    if (d > 128) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_linear_chunked_conv_workspace_bytes(B, H, Hg, Wg, d, chunk, direction, dtype);
+    if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    const long long U = (long long)B * H;
+    if (!grid_ok(U, N * d)) return TTT_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t es = dtype == TTT_BF16 ? 2 : 4;
+    char* w = static_cast<char*>(workspace);
+    void* kp = w;
+    void* vp = w + align256((size_t)U * N * d * es);
+    void* rest = w + 2 * align256((size_t)U * N * d * es);
+    const size_t rest_bytes = workspace_bytes - 2 * align256((size_t)U * N * d * es);
+    if (dtype == TTT_BF16) {
+        using T = __nv_bfloat16;
+        simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(k), wk,
+                                                                         static_cast<T*>(kp), H, Hg, Wg, d);
+        simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(v), wv,
+                                                                         static_cast<T*>(vp), H, Hg, Wg, d);
+    } else {
+        using T = float;
+        simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(k), wk,
+                                                                         static_cast<T*>(kp), H, Hg, Wg, d);
+        simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(v), wv,
+                                                                         static_cast<T*>(vp), H, Hg, Wg, d);
+    }
+    if (int rc = launched(2)) return rc;
+    return ttt_linear_chunked(q, kp, vp, w0, out, B, H, (int)N, d, chunk, eta, direction, dtype, rest, rest_bytes,
+                              stream);
 }
 
 // ------------------------------------------------------------------ no-allocation scan ---

@@ -72,6 +72,16 @@ def chunked_inputs(B, H, N, d, dtype="bf16", seed=0):
     return linear_inputs(B, H, N, d, dtype=dtype, seed=seed)
 
 
+def chunked_conv_inputs(B, H, Hg, Wg, d, dtype="bf16", seed=0):
+    """Chunked-scan inputs on an Hg x Wg grid plus the two 3x3 depthwise filters of the Conv2d
+    preprocessing: wk, wv [H,d,3,3] fp32 ~ N(0, 1/9) (drawn after W0, K's filter first)."""
+    inp = linear_inputs(B, H, Hg * Wg, d, dtype=dtype, seed=seed)
+    g = _gen(seed + 7919)
+    inp["wk"] = _randn((H, d, 3, 3), g, 1.0 / 3.0, torch.float32)
+    inp["wv"] = _randn((H, d, 3, 3), g, 1.0 / 3.0, torch.float32)
+    return inp
+
+
 # The workloads of the layer, by name.  Each entry: (kind, kwargs for the generator, eta, extra)
 CONFIGS = {
     # TTT-Linear, fp32, one 14x14 grid, one head of d = 64

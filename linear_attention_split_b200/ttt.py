@@ -51,6 +51,10 @@ def lib():
         L.ttt_kernel_launch_count.argtypes = []
         L.ttt_device_error.restype = i
         L.ttt_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.ttt_debug_set_wait_limit.restype = i
+        L.ttt_debug_set_wait_limit.argtypes = [ctypes.c_longlong]
+        L.ttt_debug_arm_fault.restype = i
+        L.ttt_debug_arm_fault.argtypes = [ctypes.c_uint]
         L.ttt_linear_fullbatch_workspace_bytes.restype = sz
         L.ttt_linear_fullbatch_workspace_bytes.argtypes = [i, i, i, i, i]
         L.ttt_linear_fullbatch.restype = i
@@ -67,6 +71,18 @@ def lib():
         L.ttt_linear_chunked_bidir_workspace_bytes.argtypes = [i, i, i, i, i, i]
         L.ttt_linear_chunked_bidir.restype = i
         L.ttt_linear_chunked_bidir.argtypes = [p, p, p, p, p, i, i, i, i, i, f, i, p, sz, p]
+        L.ttt_linear_chunked_workspace_bytes.restype = sz
+        L.ttt_linear_chunked_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.ttt_linear_chunked.restype = i
+        L.ttt_linear_chunked.argtypes = [p, p, p, p, p, i, i, i, i, i, f, i, i, p, sz, p]
+        L.ttt_linear_minibatch_workspace_bytes.restype = sz
+        L.ttt_linear_minibatch_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.ttt_linear_minibatch.restype = i
+        L.ttt_linear_minibatch.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, f, i, p, sz, p]
+        L.ttt_linear_chunked_conv_workspace_bytes.restype = sz
+        L.ttt_linear_chunked_conv_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        L.ttt_linear_chunked_conv.restype = i
+        L.ttt_linear_chunked_conv.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, f, i, i, p, sz, p]
         L.ttt_linear_chunked_bidir_noalloc.restype = i
         L.ttt_linear_chunked_bidir_noalloc.argtypes = [p, p, p, p, p, i, i, i, i, i, f, i, p]
         L.ttt_linear_chunked_bidir_noalloc_max_bytes.restype = sz
@@ -199,6 +215,61 @@ def ttt_linear_chunked_bidir(q, k, v, w0, out, chunk, eta=1.0, workspace=None, s
     return out
 
 
+def ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, direction, dtype):
+    return lib().ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, direction, dtype)
+
+
+def ttt_linear_chunked(q, k, v, w0, out, chunk, eta=1.0, direction=0, workspace=None, stream=None):
+    """One-way (direction +1 raster, -1 reverse) or bidirectional (0) chunked scan."""
+    dt = _dtype(q, k, v, out)
+    _weights(w0)
+    B, H, N, d = q.shape
+    ws, nbytes = _workspace(ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, direction, dt), workspace,
+                            q.device)
+    rc = lib().ttt_linear_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(out), B, H, N, d, int(chunk),
+                                  float(eta), int(direction), dt, _ptr(ws), nbytes, _stream(stream))
+    _check("ttt_linear_chunked", rc)
+    return out
+
+
+def ttt_linear_minibatch_workspace_bytes(B, H, N, d, chunk, epochs, dtype):
+    return lib().ttt_linear_minibatch_workspace_bytes(B, H, N, d, chunk, epochs, dtype)
+
+
+def ttt_linear_minibatch(q, k, v, w0, out, chunk, epochs=1, w_final=None, eta=1.0, workspace=None, stream=None):
+    """`epochs` epochs of mini-batch inner training (chunks of `chunk` tokens), then out = Q W_final."""
+    dt = _dtype(q, k, v, out)
+    _weights(w0, w_final)
+    B, H, N, d = q.shape
+    ws, nbytes = _workspace(ttt_linear_minibatch_workspace_bytes(B, H, N, d, chunk, epochs, dt), workspace,
+                            q.device)
+    rc = lib().ttt_linear_minibatch(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(out), _ptr(w_final), B, H, N, d,
+                                    int(chunk), int(epochs), float(eta), dt, _ptr(ws), nbytes, _stream(stream))
+    _check("ttt_linear_minibatch", rc)
+    return out
+
+
+def ttt_linear_chunked_conv_workspace_bytes(B, H, Hg, Wg, d, chunk, direction, dtype):
+    return lib().ttt_linear_chunked_conv_workspace_bytes(B, H, Hg, Wg, d, chunk, direction, dtype)
+
+
+def ttt_linear_chunked_conv(q, k, v, w0, wk, wv, out, Hg, Wg, chunk, eta=1.0, direction=0, workspace=None,
+                            stream=None):
+    """Chunked scan on (Q, conv3x3(K; wk), conv3x3(V; wv)) over the Hg x Wg token grid."""
+    dt = _dtype(q, k, v, out)
+    _weights(w0, wk, wv)
+    B, H, N, d = q.shape
+    if N != Hg * Wg:
+        raise ValueError("N must equal Hg * Wg")
+    ws, nbytes = _workspace(ttt_linear_chunked_conv_workspace_bytes(B, H, Hg, Wg, d, chunk, direction, dt),
+                            workspace, q.device)
+    rc = lib().ttt_linear_chunked_conv(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(wk), _ptr(wv), _ptr(out), B, H,
+                                       Hg, Wg, d, int(chunk), float(eta), int(direction), dt, _ptr(ws), nbytes,
+                                       _stream(stream))
+    _check("ttt_linear_chunked_conv", rc)
+    return out
+
+
 def ttt_linear_chunked_bidir_noalloc(q, k, v, w0, out, chunk, eta=1.0, stream=None):
     """The chunked scan without a workspace argument: for callers that may not allocate
     device memory at call time.  Its scratch is a fixed array inside the library's device
@@ -211,6 +282,19 @@ def ttt_linear_chunked_bidir_noalloc(q, k, v, w0, out, chunk, eta=1.0, stream=No
                                                 int(chunk), float(eta), dt, _stream(stream))
     _check("ttt_linear_chunked_bidir_noalloc", rc)
     return out
+
+
+TTT_FAULT_SKIP_LOAD = 0x1
+
+
+def debug_set_wait_limit(cycles: int) -> None:
+    """Bounded-wait limit (SM cycles) of kernels launched afterwards; <= 0 restores the default."""
+    _check("ttt_debug_set_wait_limit", lib().ttt_debug_set_wait_limit(int(cycles)))
+
+
+def debug_arm_fault(bits: int) -> None:
+    """Arm (bits != 0) or clear (0) the simulated lost-transfer test hook."""
+    _check("ttt_debug_arm_fault", lib().ttt_debug_arm_fault(int(bits)))
 
 
 def kernel_launch_count() -> int:
@@ -251,6 +335,26 @@ def mlp_fullbatch(q, k, v, w1, w2, eta=1.0, with_w_star=False):
     w2s = torch.empty((B, H, h, d), dtype=torch.float32, device=q.device) if with_w_star else None
     ttt_mlp_fullbatch(q, k, v, w1, w2, out, w1s, w2s, eta)
     return (out, w1s, w2s) if with_w_star else out
+
+
+def linear_chunked(q, k, v, w0, chunk, eta=1.0, direction=0):
+    out = torch.empty_like(q)
+    ttt_linear_chunked(q, k, v, w0, out, chunk, eta, direction)
+    return out
+
+
+def linear_minibatch(q, k, v, w0, chunk, epochs=1, eta=1.0, with_w_final=False):
+    out = torch.empty_like(q)
+    wf = torch.empty((q.shape[0], q.shape[1], q.shape[3], q.shape[3]), dtype=torch.float32,
+                     device=q.device) if with_w_final else None
+    ttt_linear_minibatch(q, k, v, w0, out, chunk, epochs, wf, eta)
+    return (out, wf) if with_w_final else out
+
+
+def linear_chunked_conv(q, k, v, w0, wk, wv, Hg, Wg, chunk, eta=1.0, direction=0):
+    out = torch.empty_like(q)
+    ttt_linear_chunked_conv(q, k, v, w0, wk, wv, out, Hg, Wg, chunk, eta, direction)
+    return out
 
 
 def linear_chunked_bidir(q, k, v, w0, chunk, eta=1.0):

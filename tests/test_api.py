@@ -16,10 +16,24 @@ def L():
     return ttt.lib()
 
 
+EXPECTED = {
+    "ttt_status_string", "ttt_version", "ttt_kernel_launch_count", "ttt_device_error",
+    "ttt_debug_set_wait_limit", "ttt_debug_arm_fault",
+    "ttt_linear_fullbatch_workspace_bytes", "ttt_linear_fullbatch",
+    "ttt_dwconv_fullbatch_workspace_bytes", "ttt_dwconv_fullbatch",
+    "ttt_mlp_fullbatch_workspace_bytes", "ttt_mlp_fullbatch",
+    "ttt_linear_chunked_bidir_workspace_bytes", "ttt_linear_chunked_bidir",
+    "ttt_linear_chunked_bidir_noalloc", "ttt_linear_chunked_bidir_noalloc_max_bytes",
+    "ttt_linear_chunked_workspace_bytes", "ttt_linear_chunked",
+    "ttt_linear_minibatch_workspace_bytes", "ttt_linear_minibatch",
+    "ttt_linear_chunked_conv_workspace_bytes", "ttt_linear_chunked_conv",
+}
+
+
 def test_exports_every_declared_symbol(L):
-    names = ttt.declared_functions()
-    assert len(names) == 14
-    for n in names:
+    names = set(ttt.declared_functions())
+    assert EXPECTED <= names, EXPECTED - names
+    for n in sorted(names):
         assert hasattr(L, n), n
 
 
@@ -105,3 +119,51 @@ def test_noalloc_scan_rejects_sizes_beyond_its_scratch(L):
     assert L.ttt_linear_chunked_bidir_noalloc_max_bytes() == 16 << 20
     rc = L.ttt_linear_chunked_bidir_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 3, 6400, 64, 64, 1.0, 1, None)
     assert rc == 3
+
+
+def test_one_way_scan_rejects_bad_arguments(L):
+    f = L.ttt_linear_chunked
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 64, 1.0, 1, 1, FAKE, 1 << 30, None]
+    for direction in (2, -2):
+        a = list(ok)
+        a[11] = direction
+        assert f(*a) == 1
+    a = list(ok)
+    a[7] = 100  # N % chunk != 0
+    assert f(*a) == 1
+    # a one-way scan on the tensor-core path needs no workspace; both directions do
+    assert L.ttt_linear_chunked_workspace_bytes(2, 3, 640, 64, 64, 1, 1) == 0
+    assert L.ttt_linear_chunked_workspace_bytes(2, 3, 640, 64, 64, 0, 1) == \
+        L.ttt_linear_chunked_bidir_workspace_bytes(2, 3, 640, 64, 64, 1) > 0
+    assert L.ttt_linear_chunked_workspace_bytes(2, 3, 640, 32, 16, -1, 0) > 0
+
+
+def test_minibatch_rejects_bad_arguments(L):
+    f = L.ttt_linear_minibatch
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 64, 2, 1.0, 1, FAKE, 1 << 30, None]
+    a = list(ok)
+    a[11] = 0  # epochs
+    assert f(*a) == 1
+    a = list(ok)
+    a[10] = 48  # 128 % 48
+    assert f(*a) == 1
+    a = list(ok)
+    a[14] = None  # the workspace is always needed
+    assert f(*a) == 3
+    assert L.ttt_linear_minibatch_workspace_bytes(2, 2, 128, 64, 64, 2, 1) >= 2 * 2 * 64 * 64 * 4
+
+
+def test_chunked_conv_rejects_bad_arguments(L):
+    f = L.ttt_linear_chunked_conv
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 8, 64, 64, 1.0, 0, 1, FAKE, 1 << 30, None]
+    a = list(ok)
+    a[4] = None  # wk
+    assert f(*a) == 1
+    a = list(ok)
+    a[12] = 48  # 64 tokens % 48
+    assert f(*a) == 1
+    a = list(ok)
+    a[17] = 16
+    assert f(*a) == 3
+    need = L.ttt_linear_chunked_conv_workspace_bytes(2, 3, 80, 80, 64, 64, 0, 1)
+    assert need >= 2 * 2 * 3 * 6400 * 64 * 2

@@ -44,3 +44,17 @@ def test_light_tailed_bf16_rounding_passes_raw_bar():
     e, raw = err(torch.tensor(ref, dtype=torch.float32).bfloat16(), ref, torch.bfloat16)
     rms = np.sqrt(np.mean(ref ** 2))
     assert e == raw and raw <= 2.0 ** (2 - 8) / rms < 2e-2
+
+
+def test_auto_floor_only_where_exact_rounding_fails_the_bar():
+    from tolerance import rounding_alone
+    rng = np.random.default_rng(2)
+    light = rng.standard_normal(100000)              # rounding alone ~1.2e-2: raw bar stands
+    heavy = rng.standard_normal(100000) ** 3         # rounding alone far above 2e-2
+    assert rounding_alone(light) < 2e-2 < rounding_alone(heavy)
+    g = torch.tensor(light, dtype=torch.float32).bfloat16()
+    e, raw = err(g, light, torch.bfloat16, rounding_floor="auto")
+    assert e == raw
+    g = torch.tensor(heavy, dtype=torch.float32).bfloat16()
+    e, raw = err(g, heavy, torch.bfloat16, rounding_floor="auto")
+    assert e < 1e-6 < raw  # exact rounding (via fp32) is all the difference there is
