@@ -95,6 +95,23 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* --------------------------------------------------------------------------------------
+ * Backward of the TTT-Linear full-batch step (outer training through the inner step: the
+ * ViT^3 abstract's "parallelizable computation"; the ViT^3 blog notes the official code writes
+ * the closed-form gradient of the inner step by hand).  For an upstream gradient dO = dL/dO of
+ * the output of ttt_linear_fullbatch, with M = Q^T dO and A = W0 M^T + M W0^T, per unit:
+ *     dQ = dO W*^T,  dV = (eta/N) K M,  dK = -(eta/N)(K A - V M^T),
+ *     dW0[h] = sum over the batch entries b of  M - (eta/N) G M   (W0 is shared per head)
+ *   q, k, v, dout, dq, dk, dv : [B, H, N, d]   dtype (dq, dk, dv are outputs)
+ *   w0 : [H, d, d] fp32;  dw0 : [H, d, d] fp32 output
+ * bf16 with d = 64 runs the tensor-core kernels, everything else the CUDA-core kernels; the
+ * workspace is always needed.  dW0 is summed over the batch in a fixed order (deterministic).
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_linear_fullbatch_bwd_workspace_bytes(int B, int H, int N, int d, int dtype);
+int ttt_linear_fullbatch_bwd(const void* q, const void* k, const void* v, const float* w0, const void* dout,
+                             void* dq, void* dk, void* dv, float* dw0, int B, int H, int N, int d, float eta,
+                             int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
  * 3x3 depthwise-conv inner model on the Hg x Wg token grid (ViT^3 blog, design study: a
  * 3x3 depthwise convolution as the visual inner module).  Per image b and channel c:
  *     F_w(X)(y, x) = sum_{a,b in 0..2} w[a][b] X(y+a-1, x+b-1)   (zero padding, no bias)

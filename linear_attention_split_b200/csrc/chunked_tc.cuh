@@ -20,8 +20,9 @@
 // plain and transposing ldmatrix.  Nothing of the recurrence goes through shared memory, and
 // no other warp takes part in it.  The step's K, Q and the CTA's 16 V
 // columns arrive through a TMA ring filled by a producer warp (warp 4).  Each step the
-// recurrence warp hands W's bf16 B fragments (2 KB) to an output warp of its direction
-// (warps 2, 3) through a small ring (wready / wfree); the output warp computes O_c = Q_c W
+// recurrence warp hands its fp32 copy of W (4 KB) to an output warp of its direction (warps
+// 2, 3) through a small ring (wready / wfree); the output warp splits it into bf16 hi + lo B
+// fragments and computes O_c = Q_c W_hi + Q_c W_lo (W kept to 2^-17 in the output)
 // and the combine of the two directions, which meet in the middle: at step s < nc/2 each
 // direction parks its fp32 partial output for its chunk in the workspace; at step s >= nc/2
 // it adds the partner's parked partial, rounds once to bf16 and stores O (deterministic).
@@ -43,7 +44,7 @@ constexpr int VT = CB * NCOL * 2;       // V columns tile: 2 KB
 constexpr int STAGE = 2 * TILE + VT;    // one direction's data for one step
 constexpr int STAGES = 3;
 constexpr int WBUF = 4;                 // depth of the W hand-over ring
-constexpr int WFR = 16 * 32 * 4;        // one W slice as B fragments: 16 registers x 32 lanes
+constexpr int WFR = 32 * 32 * 4;        // one W slice (fp32 master copy): 32 registers x 32 lanes
 constexpr int THREADS = 5 * 32;         // 2 recurrence warps, 2 output warps, producer
 constexpr int PF = 2;                   // steps ahead that the partner's partials are copied
 constexpr int PKB = CB * NCOL * 4;       // one chunk's partials for the CTA's columns (4 KB)
@@ -254,13 +255,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) wt[n][e] -= p.eta_over_b * dwt[n][e];
             make_a();
-            // ---- hand W (after this step) to the output warp -----------------------------
+            // ---- hand W (after this step, fp32) to the output warp ---------------------------
             if (!wf) mbar_wait(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             {
-                uint4* dst = wfr_ptr(dir, b);
+                float4* dst = reinterpret_cast<float4*>(wfr_ptr(dir, b));
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    dst[ks * 32 + lane] = make_uint4(wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3]);
+                for (int n = 0; n < 8; ++n) dst[n * 32 + lane] = make_float4(wt[n][0], wt[n][1], wt[n][2], wt[n][3]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->wready[dir][b]);
@@ -296,16 +296,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) load_a(qb, 0, ks, qa[ks]);
         mbar_wait(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
-        uint32_t bw[4][2][2];  // B fragments of W: k-step ks, column tile j
+        // B fragments of W as bf16 hi + lo: k-step ks, column tile j (the recurrence warp's
+        // W^T accumulator pairs, packed as its A fragments are)
+        uint32_t bw[2][4][2][2];
         {
-            const uint4* src = wfr_ptr(dir, b);
+            const float4* src = reinterpret_cast<const float4*>(wfr_ptr(dir, b));
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint4 x = src[ks * 32 + lane];
-                bw[ks][0][0] = x.x;
-                bw[ks][1][0] = x.y;
-                bw[ks][0][1] = x.z;
-                bw[ks][1][1] = x.w;
+                const float4 x = src[(2 * ks) * 32 + lane], y = src[(2 * ks + 1) * 32 + lane];
+                const float v[4][2] = {{x.x, x.y}, {x.z, x.w}, {y.x, y.y}, {y.z, y.w}};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    hi[e] = pack_bf16(v[e][0], v[e][1]);
+                    const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[e]));
+                    lo[e] = pack_bf16(v[e][0] - hf.x, v[e][1] - hf.y);
+                }
+                // A-fragment order {wa0, wa1, wa2, wa3} -> B fragments (j = 0: {0, 2}, j = 1: {1, 3})
+                bw[0][ks][0][0] = hi[0];
+                bw[0][ks][1][0] = hi[1];
+                bw[0][ks][0][1] = hi[2];
+                bw[0][ks][1][1] = hi[3];
+                bw[1][ks][0][0] = lo[0];
+                bw[1][ks][1][0] = lo[1];
+                bw[1][ks][0][1] = lo[2];
+                bw[1][ks][1][1] = lo[3];
             }
         }
         __syncwarp();
@@ -323,9 +338,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) o[i][j][e] = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
+            for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
-                for (int j = 0; j < 2; ++j) mma_bf16(o[i][j], qa[ks], bw[ks][j][0], bw[ks][j][1]);
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) mma_bf16(o[i][j], qa[ks], bw[hl][ks][j][0], bw[hl][ks][j][1]);
             if (i < 3) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)

@@ -1,0 +1,403 @@
+// linear_bwd_tc.cuh -- backward of the TTT-Linear full-batch step on the tcgen05 tensor cores,
+// bf16, d = 64 (outer training through the inner step).
+//
+// Operation: the layer ("ViT^3" blog, steps 1-3; TTT-Linear of the TTT abstract) is, per unit,
+//     W* = W0 - (eta/N)(G W0 - C),  G = K^T K,  C = K^T V,   O = Q W*,
+// and for an upstream gradient dO the chain rule gives (M = Q^T dO, A = W0 M^T + M W0^T):
+//     dQ = dO W*^T,   dV = (eta/N) K M,   dK = -(eta/N)(K A - V M^T),
+//     dW0 = sum over the batch entries of a head of  M - (eta/N) G M.
+// The gradient of the inner step is written by hand, as the ViT^3 blog notes the official code
+// does ("从官方代码看…", third point).  Four launches:
+//   reduce : CTAs split each unit's tokens (as the forward does); per tile of V, K, Q, dO two
+//            tcgen05 MMAs accumulate [V | K]^T K (C^T and G) and [Q | dO]^T dO (M in its first
+//            64 rows) in TMEM; each CTA writes its partial G, C^T, M (fp32) to the workspace.
+//   finish : one block per unit adds the partials in split order (deterministic) and forms, in
+//            fp32 on the CUDA cores, W*, A and dW0_u; it writes the four d x d right-hand
+//            operands of the token pass -- W*, (eta/N) M^T, -(eta/N) A, (eta/N) M -- each as bf16
+//            hi + lo (row-major rows = output columns, i.e. K-major for the MMA).
+//   apply  : per tile of dO, K, V: dQ = dO W*, dV = K (eta/N) M^T-operand, dK = K (-eta/N A) +
+//            V (eta/N M), each product taken as hi + lo into one 64-column TMEM accumulator;
+//            the outputs are written as bf16 over the consumed input tiles and stored by TMA.
+//   dw0    : dW0[h] = sum_b dW0_(b,h) in batch order (the CUDA-core kernel of simt.cuh).
+// Every wait is bounded (common.cuh).
+#pragma once
+#include "common.cuh"
+
+namespace lbw {
+
+constexpr int D = 64;
+constexpr int ROWB = 128;                 // bytes per token row (64 bf16)
+constexpr int MT = 128;                   // rows reserved per tile (TT <= MT are used)
+constexpr int TILE = MT * ROWB;           // 16 KB
+constexpr int OP = D * ROWB;              // one 64 x 64 bf16 K-major operand, 8 KB
+constexpr int DD = D * D;
+
+// ----------------------------------------------------------------------------- reduce ----
+constexpr int R_STAGES = 3;
+constexpr int R_STAGE = 4 * TILE;         // V, K, Q, dO
+constexpr int R_THREADS = 64 + 128;       // producer, issuer, 4 epilogue warps
+constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);  // A MN-major, B MN-major
+constexpr uint32_t IDESC_N64 = tc::idesc_bf16(128, 64, 0, 0);   // A K-major, B K-major
+
+struct RParams {
+    float* part;      // [U][S][3][64][64]: G, C^T, M
+    int TT, n_tiles;  // token rows per tile, tiles per unit
+};
+struct RBars {
+    uint64_t full[R_STAGES], empty[R_STAGES], done;
+    uint32_t tmem_base;
+};
+constexpr int r_smem_bytes() { return R_STAGES * R_STAGE + (int)sizeof(RBars) + 1024; }
+
+__global__ void __launch_bounds__(R_THREADS, 1)
+    reduce_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g, const RParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    RBars* bars = reinterpret_cast<RBars*>(ring + R_STAGES * R_STAGE);
+    const int S = gridDim.x, r = blockIdx.x, u = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int TT = p.TT;
+    const int n_t = r < p.n_tiles ? (p.n_tiles - r + S - 1) / S : 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < R_STAGES; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->done, 1);
+        mbar_fence_init();
+    }
+    if (warp == 1) tc::alloc(&bars->tmem_base, 128);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_g);
+            for (int i = 0; i < n_t; ++i) {
+                const int slot = i % R_STAGES, use = i / R_STAGES;
+                if (use > 0) mbar_wait(&bars->empty[slot], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                uint8_t* dst = ring + slot * R_STAGE;
+                const int row = (r + i * S) * TT;
+                mbar_expect_tx(&bars->full[slot], 4 * TT * ROWB);
+                tma_load_3d(dst, &tm_v, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + TILE, &tm_k, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + 2 * TILE, &tm_q, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + 3 * TILE, &tm_g, 0, row, u, &bars->full[slot]);
+                if (i == R_STAGES - 1)  // the rest of this CTA's tiles into L2 now
+                    for (int j = R_STAGES; j < n_t; ++j) {
+                        const int rj = (r + j * S) * TT;
+                        tma_prefetch_l2_3d(&tm_v, 0, rj, u);
+                        tma_prefetch_l2_3d(&tm_k, 0, rj, u);
+                        tma_prefetch_l2_3d(&tm_q, 0, rj, u);
+                        tma_prefetch_l2_3d(&tm_g, 0, rj, u);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int i = 0; i < n_t; ++i) {
+                const int slot = i % R_STAGES;
+                mbar_wait(&bars->full[slot], (i / R_STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                const uint32_t vb = smem_u32(ring + slot * R_STAGE);
+                // [V | K]^T K and [Q | dO]^T dO: A MN-major over two adjacent tiles (LBO), B MN-major
+                const uint64_t a1 = tc::smem_desc(vb, TILE, 1024, 2), b1 = tc::smem_desc(vb + TILE, TILE, 1024, 2);
+                const uint64_t a2 = tc::smem_desc(vb + 2 * TILE, TILE, 1024, 2);
+                const uint64_t b2 = tc::smem_desc(vb + 3 * TILE, TILE, 1024, 2);
+                for (int ks = 0; ks < TT / 16; ++ks) {
+                    const int acc = (i > 0 || ks > 0) ? 1 : 0;
+                    tc::mma_bf16(tmem, a1 + (uint64_t)(ks * 128), b1 + (uint64_t)(ks * 128), IDESC_GRAM, acc);
+                    tc::mma_bf16(tmem + 64, a2 + (uint64_t)(ks * 128), b2 + (uint64_t)(ks * 128), IDESC_GRAM, acc);
+                }
+                tc::commit(&bars->empty[slot]);
+            }
+            tc::commit(&bars->done);
+        }
+    } else {
+        // lane row: rows 0-63 hold C^T (first accumulator) and M (second), rows 64-127 hold G
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        float* part = p.part + ((size_t)u * S + r) * 3 * DD;
+        if (n_t > 0) {
+            mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
+            tc::fence_after();
+        }
+#pragma unroll
+        for (int acc = 0; acc < 2; ++acc) {
+            if (acc == 1 && row >= D) break;  // rows 64-127 of [Q | dO]^T dO are not needed
+            float* dst = acc == 0 ? (row >= D ? part + (row - D) * D : part + DD + row * D) : part + 2 * DD + row * D;
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                float x[16];
+                if (n_t > 0) {
+                    tc::ld16(lane_base + acc * 64 + c16 * 16, x);
+                    tc::wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4*>(dst + c16 * 16 + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            }
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 1) tc::dealloc(tmem, 128);
+}
+
+// ----------------------------------------------------------------------------- finish ----
+struct FParams {
+    const float* part;     // [U][S][3][64][64]
+    const float* w0;       // [H][64][64]
+    __nv_bfloat16* ops;    // [U][8][64][64]: W* hi/lo, (eta/N) M^T hi/lo, -(eta/N) A hi/lo, (eta/N) M hi/lo
+    float* dw0u;           // [U][64][64]
+    int H, S;
+    float eta_over_n;
+};
+constexpr int FP = D + 1;  // padded row of the shared-memory matrices
+constexpr int f_smem_bytes() { return 5 * D * FP * 4; }
+
+__device__ __forceinline__ void put_hilo(__nv_bfloat16* ops, int m, int row, int col, float x) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    ops[(m * D + row) * D + col] = hi;
+    ops[((m + 1) * D + row) * D + col] = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+__global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
+    extern __shared__ float fsm[];
+    float* Gs = fsm;
+    float* Cts = Gs + D * FP;  // C^T
+    float* Ms = Cts + D * FP;
+    float* W0s = Ms + D * FP;
+    float* Xs = W0s + D * FP;  // W0 M^T
+    const int u = blockIdx.x, tid = threadIdx.x;
+    const float* W0 = p.w0 + (size_t)(u % p.H) * DD;
+    for (int e = tid; e < DD; e += 256) {
+        float g = 0.f, ct = 0.f, m = 0.f;
+        for (int s = 0; s < p.S; ++s) {  // split order
+            const float* b = p.part + ((size_t)u * p.S + s) * 3 * DD;
+            g += b[e];
+            ct += b[DD + e];
+            m += b[2 * DD + e];
+        }
+        const int r = e >> 6, c = e & 63;
+        Gs[r * FP + c] = g;
+        Cts[r * FP + c] = ct;
+        Ms[r * FP + c] = m;
+        W0s[r * FP + c] = W0[e];
+    }
+    __syncthreads();
+    const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
+    float gw[4][4] = {}, x[4][4] = {}, gm[4][4] = {};
+    for (int k = 0; k < D; ++k) {
+        float gr[4], wr[4], wc[4], mt[4], mk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            gr[i] = Gs[(r0 + i) * FP + k];
+            wr[i] = W0s[(r0 + i) * FP + k];
+            wc[i] = W0s[k * FP + c0 + i];
+            mt[i] = Ms[(c0 + i) * FP + k];
+            mk[i] = Ms[k * FP + c0 + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                gw[i][j] = fmaf(gr[i], wc[j], gw[i][j]);  // (G W0)[r][c]
+                x[i][j] = fmaf(wr[i], mt[j], x[i][j]);    // (W0 M^T)[r][c]
+                gm[i][j] = fmaf(gr[i], mk[j], gm[i][j]);  // (G M)[r][c]
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Xs[(r0 + i) * FP + c0 + j] = x[i][j];
+    __syncthreads();
+    __nv_bfloat16* ops = p.ops + (size_t)u * 8 * DD;
+    const float en = p.eta_over_n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = r0 + i, c = c0 + j;
+            const float ws = W0s[r * FP + c] - en * (gw[i][j] - Cts[c * FP + r]);  // C[r][c] = C^T[c][r]
+            const float a = Xs[r * FP + c] + Xs[c * FP + r];
+            const float m = Ms[r * FP + c];
+            p.dw0u[(size_t)u * DD + r * D + c] = m - en * gm[i][j];
+            put_hilo(ops, 0, r, c, ws);        // dQ[t][c'] = sum_b dO[t][b] W*[c'][b]
+            put_hilo(ops, 2, c, r, en * m);    // dV[t][c'] = sum_a K[t][a] (eta/N) M[a][c']
+            put_hilo(ops, 4, r, c, -en * a);   // dK[t][c'] += sum_a K[t][a] (-eta/N) A[a][c']  (A symmetric)
+            put_hilo(ops, 6, r, c, en * m);    // dK[t][c'] += sum_b V[t][b] (eta/N) M[c'][b]
+        }
+}
+
+// ----------------------------------------------------------------------------- apply -----
+constexpr int A_STAGES = 3;
+constexpr int A_STAGE = 3 * TILE;         // dO, K, V (dQ, dK, dV are written over them)
+constexpr int OPS = 8 * OP;               // the eight right-hand operands, 64 KB
+constexpr int A_EPI_WARPS = 8;
+constexpr int A_THREADS = 64 + 32 * A_EPI_WARPS;
+
+struct AParams {
+    int TT, n_tiles;
+};
+struct ABars {
+    uint64_t opfull, full[A_STAGES], empty[A_STAGES], tfull[2], tempty[2];
+    uint32_t tmem_base;
+};
+constexpr int a_smem_bytes() { return OPS + A_STAGES * A_STAGE + (int)sizeof(ABars) + 1024; }
+
+__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
+
+__global__ void __launch_bounds__(A_THREADS, 1)
+    apply_kernel(const __grid_constant__ CUtensorMap tm_ops, const __grid_constant__ CUtensorMap tm_g,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                 const __grid_constant__ CUtensorMap tm_dv, const AParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ops = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = ops + OPS;
+    ABars* bars = reinterpret_cast<ABars*>(ring + A_STAGES * A_STAGE);
+    const int S = gridDim.x, r = blockIdx.x, u = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int TT = p.TT;
+    const int n_t = r < p.n_tiles ? (p.n_tiles - r + S - 1) / S : 0;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->opfull, 1);
+        for (int s = 0; s < A_STAGES; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->tfull[b], 1);
+            mbar_init(&bars->tempty[b], A_EPI_WARPS / 2);
+        }
+        mbar_fence_init();
+    }
+    if (warp == 1) tc::alloc(&bars->tmem_base, 512);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_ops);
+            tma_prefetch_desc(&tm_g);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_expect_tx(&bars->opfull, OPS);
+            for (int m = 0; m < 8; ++m) tma_load_3d(ops + m * OP, &tm_ops, 0, m * D, u, &bars->opfull);
+            for (int i = 0; i < n_t; ++i) {
+                const int slot = i % A_STAGES, use = i / A_STAGES;
+                if (use > 0) mbar_wait(&bars->empty[slot], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                uint8_t* dst = ring + slot * A_STAGE;
+                const int row = (r + i * S) * TT;
+                mbar_expect_tx(&bars->full[slot], 3 * TT * ROWB);
+                tma_load_3d(dst, &tm_g, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + TILE, &tm_k, 0, row, u, &bars->full[slot]);
+                tma_load_3d(dst + 2 * TILE, &tm_v, 0, row, u, &bars->full[slot]);
+                if (i == A_STAGES - 1)
+                    for (int j = A_STAGES; j < n_t; ++j) {
+                        const int rj = (r + j * S) * TT;
+                        tma_prefetch_l2_3d(&tm_g, 0, rj, u);
+                        tma_prefetch_l2_3d(&tm_k, 0, rj, u);
+                        tma_prefetch_l2_3d(&tm_v, 0, rj, u);
+                    }
+            }
+            mbar_wait(&bars->opfull, 0, TTT_DEVERR_TIMEOUT_TMA);  // no load in flight at exit
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && n_t > 0) {
+            mbar_wait(&bars->opfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+            const uint32_t ob = smem_u32(ops);
+            uint64_t od[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) od[m] = tc::smem_desc(ob + m * OP, 16, 1024, 2);
+            for (int t = 0; t < n_t; ++t) {
+                const int b = t & 1, slot = t % A_STAGES;
+                if (t >= 2) mbar_wait(&bars->tempty[b], ((t >> 1) - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                mbar_wait(&bars->full[slot], (t / A_STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                const uint32_t sb = smem_u32(ring + slot * A_STAGE);
+                const uint64_t dg = tc::smem_desc(sb, 16, 1024, 2);
+                const uint64_t dk = tc::smem_desc(sb + TILE, 16, 1024, 2);
+                const uint64_t dv = tc::smem_desc(sb + 2 * TILE, 16, 1024, 2);
+                const uint32_t acc0 = tmem + b * 256;
+                // dQ (columns 0-63), dV (64-127), dK (128-191); each right operand as hi + lo
+#pragma unroll
+                for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const int acc = (hl > 0 || ks > 0) ? 1 : 0;
+                        tc::mma_bf16(acc0, dg + 2 * ks, od[0 + hl] + 2 * ks, IDESC_N64, acc);
+                        tc::mma_bf16(acc0 + 64, dk + 2 * ks, od[2 + hl] + 2 * ks, IDESC_N64, acc);
+                        tc::mma_bf16(acc0 + 128, dk + 2 * ks, od[4 + hl] + 2 * ks, IDESC_N64, acc);
+                    }
+#pragma unroll
+                for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) tc::mma_bf16(acc0 + 128, dv + 2 * ks, od[6 + hl] + 2 * ks, IDESC_N64, 1);
+                tc::commit(&bars->tfull[b]);
+            }
+        }
+    } else {
+        const int q4 = warp & 3;
+        const int grp = (warp - 2) >> 2;  // tile group: tiles grp, grp + 2, ...
+        const int row = q4 * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        const bool storer = (q4 == 0 && lane == 0);
+        for (int t = grp; t < n_t; t += 2) {
+            const int b = t & 1, slot = t % A_STAGES;
+            uint8_t* st = ring + slot * A_STAGE;
+            mbar_wait(&bars->tfull[b], (t >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            tc::fence_after();
+            // accumulator j -> tile: dQ over dO (tile 0), dV over V (tile 2), dK over K (tile 1)
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                uint8_t* tile = st + (j == 0 ? 0 : j == 1 ? 2 * TILE : TILE);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float o[32];
+                    tc::ld16(lane_base + b * 256 + j * 64 + half * 32, &o[0]);
+                    tc::ld16(lane_base + b * 256 + j * 64 + half * 32 + 16, &o[16]);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(tile + swz<3>((uint32_t)row * ROWB + half * 64 + c * 16)) =
+                            make_uint4(pack_bf16(o[8 * c], o[8 * c + 1]), pack_bf16(o[8 * c + 2], o[8 * c + 3]),
+                                       pack_bf16(o[8 * c + 4], o[8 * c + 5]), pack_bf16(o[8 * c + 6], o[8 * c + 7]));
+                }
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tempty[b]);
+            fence_proxy_async_smem();
+            group_sync(grp);  // all 128 rows of the three output tiles are written
+            if (storer) {
+                const int grow = (r + t * S) * TT;  // rows >= N are clipped
+                tma_store_3d(&tm_dq, 0, grow, u, st);
+                tma_store_3d(&tm_dk, 0, grow, u, st + TILE);
+                tma_store_3d(&tm_dv, 0, grow, u, st + 2 * TILE);
+                tma_store_commit();
+                tma_store_wait_read_all();  // the stage may be refilled
+                mbar_arrive(&bars->empty[slot]);
+            }
+        }
+        if (storer) tma_store_wait_all();
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 1) tc::dealloc(tmem, 512);
+}
+
+}  // namespace lbw

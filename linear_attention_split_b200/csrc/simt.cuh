@@ -356,6 +356,96 @@ __global__ void __launch_bounds__(TPB) minibatch_train(const T* __restrict__ k, 
     }
 }
 
+// ------------------------------------------------------------------ TTT-Linear backward -
+// Gradients of an outer loss through the full-batch step, for the upstream gradient dO:
+//   M = Q^T dO,  W* = W0 - (eta/N)(G W0 - C),  A = W0 M^T + M W0^T (symmetric)
+//   dQ = dO W*^T,  dV = (eta/N) K M,  dK = -(eta/N) (K A - V M^T),  dW0_u = M - (eta/N) G M
+// (the chain rule back through o = q W*, W* = W0 - eta gW, gW = (1/N) sum k^T (k W0 - v)).
+// gcm[u] = {G, C, M}, d x d each, token sums in fp64.
+template <typename T>
+__global__ void __launch_bounds__(TPB) linear_bwd_gram(const T* __restrict__ q, const T* __restrict__ k,
+                                                       const T* __restrict__ v, const T* __restrict__ g,
+                                                       float* __restrict__ gcm, int N, int d) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    const int dd = d * d;
+    if (e >= 3 * dd) return;
+    const int which = e / dd, r = (e % dd) / d, c = e % d;
+    const T* a = (which == 2 ? q : k) + u * N * d;
+    const T* b = (which == 0 ? k : which == 1 ? v : g) + u * N * d;
+    double acc = 0.0;
+    for (int t = 0; t < N; ++t)
+        acc = fma((double)to_f(a[(long long)t * d + r]), (double)to_f(b[(long long)t * d + c]), acc);
+    gcm[u * 3 * dd + e] = (float)acc;
+}
+
+// Per element (r, c) of unit u: wsa[u] = {W*, A}, dw0u[u] = dW0_u (fp32).
+__global__ void __launch_bounds__(TPB) linear_bwd_finish(const float* __restrict__ gcm, const float* __restrict__ w0,
+                                                         float* __restrict__ wsa, float* __restrict__ dw0u, int H,
+                                                         int d, float eta_over_n) {
+    const long long u = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    const int dd = d * d;
+    if (e >= dd) return;
+    const int r = e / d, c = e % d;
+    const float* G = gcm + u * 3 * dd;
+    const float* C = G + dd;
+    const float* M = C + dd;
+    const float* W0 = w0 + (u % H) * dd;
+    float gw = 0.f, xrc = 0.f, xcr = 0.f, gm = 0.f;
+    for (int m = 0; m < d; ++m) {
+        gw = fmaf(G[r * d + m], W0[m * d + c], gw);
+        xrc = fmaf(W0[r * d + m], M[c * d + m], xrc);
+        xcr = fmaf(W0[c * d + m], M[r * d + m], xcr);
+        gm = fmaf(G[r * d + m], M[m * d + c], gm);
+    }
+    wsa[u * 2 * dd + e] = W0[e] - eta_over_n * (gw - C[e]);
+    wsa[u * 2 * dd + dd + e] = xrc + xcr;
+    dw0u[u * dd + e] = M[e] - eta_over_n * gm;
+}
+
+// dQ, dK, dV at element (t, c)
+template <typename T>
+__global__ void __launch_bounds__(TPB) linear_bwd_apply(const T* __restrict__ k, const T* __restrict__ v,
+                                                        const T* __restrict__ g, const float* __restrict__ gcm,
+                                                        const float* __restrict__ wsa, T* __restrict__ dq,
+                                                        T* __restrict__ dk, T* __restrict__ dv, int N, int d,
+                                                        float eta_over_n) {
+    const long long u = blockIdx.x;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;
+    if (e >= (long long)N * d) return;
+    const long long t = e / d;
+    const int c = (int)(e % d);
+    const int dd = d * d;
+    const float* M = gcm + u * 3 * dd + 2 * dd;
+    const float* W = wsa + u * 2 * dd;
+    const float* A = W + dd;
+    const long long row = u * N * d + t * d;
+    float sq = 0.f, sv = 0.f, ska = 0.f, skv = 0.f;
+    for (int m = 0; m < d; ++m) {
+        const float gm = to_f(g[row + m]), km = to_f(k[row + m]), vm = to_f(v[row + m]);
+        sq = fmaf(gm, W[c * d + m], sq);   // dO W*^T
+        sv = fmaf(km, M[m * d + c], sv);   // K M
+        ska = fmaf(km, A[m * d + c], ska); // K A
+        skv = fmaf(vm, M[c * d + m], skv); // V M^T
+    }
+    dq[row + c] = from_f<T>(sq);
+    dv[row + c] = from_f<T>(eta_over_n * sv);
+    dk[row + c] = from_f<T>(-eta_over_n * (ska - skv));
+}
+
+// dW0[h] = sum over batch entries b (in order) of dW0_(b, h)
+__global__ void __launch_bounds__(TPB) linear_bwd_dw0(const float* __restrict__ dw0u, float* __restrict__ dw0, int B,
+                                                      int H, int d) {
+    const int h = blockIdx.x;
+    const int e = blockIdx.y * TPB + threadIdx.x;
+    const int dd = d * d;
+    if (e >= dd) return;
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += dw0u[((long long)b * H + h) * dd + e];
+    dw0[(long long)h * dd + e] = s;
+}
+
 // ------------------------------------------------------------------ conv preprocessing --
 // x' = 3x3 depthwise conv of x over the Hg x Wg token grid of each unit (zero padding, no
 // bias): one filter per feature of each head, taps w [H][d][3][3]; x, y [U][Hg*Wg][d].

@@ -17,6 +17,7 @@
 #include "simt.cuh"
 #include "linear_tc.cuh"
 #include "linear_tc5.cuh"
+#include "linear_bwd_tc.cuh"
 #include "dwconv_fused.cuh"
 #include "chunked_tc.cuh"
 #include "mlp_tc.cuh"
@@ -262,6 +263,112 @@ int linear_tc5(const void* q, const void* k, const void* v, const float* w0, voi
     cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, to, p) != cudaSuccess) return TTT_ERR_CUDA;
     return launched(1);
+}
+
+// ------------------------------------------------------------------ TTT-Linear backward
+bool linear_bwd_tc_ok(int d, int dtype) { return dtype == TTT_BF16 && d == lbw::D; }
+
+struct BwdPlan {
+    int S, TT, n_tiles;
+};
+// token splits per unit (one CTA per SM) and equal tiles of TT <= 128 rows, as in the forward
+BwdPlan bwd_plan(long long U, int N, int sms) {
+    BwdPlan b;
+    const int t128 = (N + lbw::MT - 1) / lbw::MT;
+    b.S = 1;
+    while (b.S < 8 && U * b.S * 2 <= sms && b.S * 2 <= t128) b.S *= 2;
+    const int per_cta = (N + b.S - 1) / b.S;
+    const int k_tiles = (per_cta + lbw::MT - 1) / lbw::MT;
+    b.TT = ((per_cta + k_tiles - 1) / k_tiles + 15) / 16 * 16;
+    b.n_tiles = (N + b.TT - 1) / b.TT;
+    return b;
+}
+size_t bwd_tc_ws(long long U, int S) {
+    return align256((size_t)U * S * 3 * lbw::DD * 4) + align256((size_t)U * 8 * lbw::DD * 2) +
+           align256((size_t)U * lbw::DD * 4);
+}
+size_t bwd_simt_ws(long long U, int d) {
+    return align256((size_t)U * 3 * d * d * 4) + align256((size_t)U * 2 * d * d * 4) + align256((size_t)U * d * d * 4);
+}
+
+int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, const void* g, void* dq, void* dk,
+                  void* dv, float* dw0, int B, int H, int N, float eta, void* ws, cudaStream_t st) {
+    DeviceInfo* dev = nullptr;
+    if (int rc = current_device(&dev)) return rc;
+    const long long U = (long long)B * H;
+    if (U > 65535) return TTT_ERR_UNSUPPORTED;
+    const BwdPlan pl = bwd_plan(U, N, dev->sms);
+    if (lbw::r_smem_bytes() > dev->smem_optin || lbw::a_smem_bytes() > dev->smem_optin ||
+        lbw::f_smem_bytes() > dev->smem_optin)
+        return TTT_ERR_UNSUPPORTED;
+    char* w = static_cast<char*>(ws);
+    float* part = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * pl.S * 3 * lbw::DD * 4);
+    __nv_bfloat16* ops = reinterpret_cast<__nv_bfloat16*>(w);
+    w += align256((size_t)U * 8 * lbw::DD * 2);
+    float* dw0u = reinterpret_cast<float*>(w);
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    CUtensorMap tv, tk, tq, tg, tops, tdq, tdk, tdv;
+    if (!tmap_bf16_3d(&tv, v, 64, N, (int)U, pl.TT, sw) || !tmap_bf16_3d(&tk, k, 64, N, (int)U, pl.TT, sw) ||
+        !tmap_bf16_3d(&tq, q, 64, N, (int)U, pl.TT, sw) || !tmap_bf16_3d(&tg, g, 64, N, (int)U, pl.TT, sw) ||
+        !tmap_bf16_3d(&tdq, dq, 64, N, (int)U, pl.TT, sw) || !tmap_bf16_3d(&tdk, dk, 64, N, (int)U, pl.TT, sw) ||
+        !tmap_bf16_3d(&tdv, dv, 64, N, (int)U, pl.TT, sw) ||
+        !tmap_bf16_box(&tops, ops, 64, 8 * 64, (int)U, 64, 64, sw))
+        return TTT_ERR_CUDA;
+    if (cudaFuncSetAttribute(lbw::reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lbw::r_smem_bytes()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(lbw::finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lbw::f_smem_bytes()) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(lbw::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lbw::a_smem_bytes()) !=
+            cudaSuccess)
+        return TTT_ERR_CUDA;
+    lbw::RParams rp;
+    rp.part = part;
+    rp.TT = pl.TT;
+    rp.n_tiles = pl.n_tiles;
+    lbw::reduce_kernel<<<dim3(pl.S, (unsigned)U), lbw::R_THREADS, lbw::r_smem_bytes(), st>>>(tv, tk, tq, tg, rp);
+    lbw::FParams fp;
+    fp.part = part;
+    fp.w0 = w0;
+    fp.ops = ops;
+    fp.dw0u = dw0u;
+    fp.H = H;
+    fp.S = pl.S;
+    fp.eta_over_n = (float)((double)eta / (double)N);
+    lbw::finish_kernel<<<(unsigned)U, 256, lbw::f_smem_bytes(), st>>>(fp);
+    lbw::AParams ap;
+    ap.TT = pl.TT;
+    ap.n_tiles = pl.n_tiles;
+    lbw::apply_kernel<<<dim3(pl.S, (unsigned)U), lbw::A_THREADS, lbw::a_smem_bytes(), st>>>(tops, tg, tk, tv, tdq,
+                                                                                             tdk, tdv, ap);
+    simt::linear_bwd_dw0<<<dim3((unsigned)H, (lbw::DD + simt::TPB - 1) / simt::TPB), simt::TPB, 0, st>>>(dw0u, dw0, B,
+                                                                                                       H, lbw::D);
+    return launched(4);
+}
+
+template <typename T>
+int linear_bwd_simt(const void* q, const void* k, const void* v, const float* w0, const void* g, void* dq, void* dk,
+                    void* dv, float* dw0, int B, int H, int N, int d, float eta, void* ws, cudaStream_t st) {
+    const long long U = (long long)B * H;
+    if (!grid_ok(U, 3LL * d * d) || !grid_ok(U, (long long)N * d) || !grid_ok(H, (long long)d * d))
+        return TTT_ERR_UNSUPPORTED;
+    char* w = static_cast<char*>(ws);
+    float* gcm = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * 3 * d * d * 4);
+    float* wsa = reinterpret_cast<float*>(w);
+    w += align256((size_t)U * 2 * d * d * 4);
+    float* dw0u = reinterpret_cast<float*>(w);
+    const float eta_over_n = (float)((double)eta / (double)N);
+    simt::linear_bwd_gram<T><<<grid_units(U, 3LL * d * d), simt::TPB, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(g), gcm,
+        N, d);
+    simt::linear_bwd_finish<<<grid_units(U, (long long)d * d), simt::TPB, 0, st>>>(gcm, w0, wsa, dw0u, H, d,
+                                                                                   eta_over_n);
+    simt::linear_bwd_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(g), gcm, wsa, static_cast<T*>(dq),
+        static_cast<T*>(dk), static_cast<T*>(dv), N, d, eta_over_n);
+    simt::linear_bwd_dw0<<<grid_units(H, (long long)d * d), simt::TPB, 0, st>>>(dw0u, dw0, B, H, d);
+    return launched(4);
 }
 
 int check_common(const void* q, const void* k, const void* v, const void* out, int dtype, float eta) {
@@ -662,6 +769,36 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
         return linear_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
     }
     return linear_simt<float>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
+}
+
+// ------------------------------------------------------------------ TTT-Linear backward
+size_t ttt_linear_fullbatch_bwd_workspace_bytes(int B, int H, int N, int d, int dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+    const long long U = (long long)B * H;
+    if (linear_bwd_tc_ok(d, dtype)) {
+        DeviceInfo* dev = nullptr;
+        const int sms = current_device(&dev) == TTT_OK ? dev->sms : 148;
+        return bwd_tc_ws(U, bwd_plan(U, N, sms).S);
+    }
+    return bwd_simt_ws(U, d);
+}
+
+int ttt_linear_fullbatch_bwd(const void* q, const void* k, const void* v, const float* w0, const void* dout,
+                             void* dq, void* dk, void* dv, float* dw0, int B, int H, int N, int d, float eta,
+                             int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    if (int rc = check_common(q, k, v, dout, dtype, eta)) return rc;
+    if (!dq || !dk || !dv || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return TTT_ERR_INVALID_ARG;
+    if (!w0 || !dw0 || !aligned16(w0) || !aligned16(dw0)) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return TTT_ERR_INVALID_ARG;
+    if (d > 128) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dtype);
+    if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (linear_bwd_tc_ok(d, dtype))
+        return linear_bwd_tc(q, k, v, w0, dout, dq, dk, dv, dw0, B, H, N, eta, workspace, st);
+    if (dtype == TTT_BF16)
+        return linear_bwd_simt<__nv_bfloat16>(q, k, v, w0, dout, dq, dk, dv, dw0, B, H, N, d, eta, workspace, st);
+    return linear_bwd_simt<float>(q, k, v, w0, dout, dq, dk, dv, dw0, B, H, N, d, eta, workspace, st);
 }
 
 // ------------------------------------------------------------------ depthwise conv ----

@@ -72,6 +72,15 @@ def chunked_inputs(B, H, N, d, dtype="bf16", seed=0):
     return linear_inputs(B, H, N, d, dtype=dtype, seed=seed)
 
 
+def linear_bwd_inputs(B, H, N, d, dtype="bf16", seed=0):
+    """The TTT-Linear inputs plus an upstream gradient dO [B,H,N,d] ~ N(0,1)/sqrt(d) in `dtype`
+    (drawn from its own stream after the layer's inputs)."""
+    inp = linear_inputs(B, H, N, d, dtype=dtype, seed=seed)
+    g = _gen(seed + 104729)
+    inp["dout"] = _randn((B, H, N, d), g, 1.0 / math.sqrt(d), DTYPES[dtype])
+    return inp
+
+
 def chunked_conv_inputs(B, H, Hg, Wg, d, dtype="bf16", seed=0):
     """Chunked-scan inputs on an Hg x Wg grid plus the two 3x3 depthwise filters of the Conv2d
     preprocessing: wk, wv [H,d,3,3] fp32 ~ N(0, 1/9) (drawn after W0, K's filter first)."""

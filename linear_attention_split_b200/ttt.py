@@ -59,6 +59,10 @@ def lib():
         L.ttt_linear_fullbatch_workspace_bytes.argtypes = [i, i, i, i, i]
         L.ttt_linear_fullbatch.restype = i
         L.ttt_linear_fullbatch.argtypes = [p, p, p, p, p, p, i, i, i, i, f, i, p, sz, p]
+        L.ttt_linear_fullbatch_bwd_workspace_bytes.restype = sz
+        L.ttt_linear_fullbatch_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.ttt_linear_fullbatch_bwd.restype = i
+        L.ttt_linear_fullbatch_bwd.argtypes = [p, p, p, p, p, p, p, p, p, i, i, i, i, f, i, p, sz, p]
         L.ttt_dwconv_fullbatch_workspace_bytes.restype = sz
         L.ttt_dwconv_fullbatch_workspace_bytes.argtypes = [i, i, i, i, i]
         L.ttt_dwconv_fullbatch.restype = i
@@ -161,6 +165,23 @@ def ttt_linear_fullbatch(q, k, v, w0, out, w_star=None, eta=1.0, workspace=None,
                                     d, float(eta), dt, _ptr(ws), nbytes, _stream(stream))
     _check("ttt_linear_fullbatch", rc)
     return out
+
+
+def ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dtype):
+    return lib().ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dtype)
+
+
+def ttt_linear_fullbatch_bwd(q, k, v, w0, dout, dq, dk, dv, dw0, eta=1.0, workspace=None, stream=None):
+    """Gradients of the full-batch TTT-Linear layer: dq, dk, dv [B,H,N,d] (dtype of q), dw0 [H,d,d] fp32."""
+    dt = _dtype(q, k, v, dout, dq, dk, dv)
+    _weights(w0, dw0)
+    B, H, N, d = q.shape
+    ws, nbytes = _workspace(ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dt), workspace, q.device)
+    rc = lib().ttt_linear_fullbatch_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w0), _ptr(dout), _ptr(dq), _ptr(dk),
+                                        _ptr(dv), _ptr(dw0), B, H, N, d, float(eta), dt, _ptr(ws), nbytes,
+                                        _stream(stream))
+    _check("ttt_linear_fullbatch_bwd", rc)
+    return dq, dk, dv, dw0
 
 
 def ttt_dwconv_fullbatch_workspace_bytes(B, Hg, Wg, C, dtype):
@@ -317,6 +338,12 @@ def linear_fullbatch(q, k, v, w0, eta=1.0, with_w_star=False):
                      device=q.device) if with_w_star else None
     ttt_linear_fullbatch(q, k, v, w0, out, ws, eta)
     return (out, ws) if with_w_star else out
+
+
+def linear_fullbatch_bwd(q, k, v, w0, dout, eta=1.0):
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dw0 = torch.empty_like(w0)
+    return ttt_linear_fullbatch_bwd(q, k, v, w0, dout, dq, dk, dv, dw0, eta)
 
 
 def dwconv_fullbatch(q, k, v, w0, eta=1.0, with_w_star=False):

@@ -27,6 +27,7 @@ EXPECTED = {
     "ttt_linear_chunked_workspace_bytes", "ttt_linear_chunked",
     "ttt_linear_minibatch_workspace_bytes", "ttt_linear_minibatch",
     "ttt_linear_chunked_conv_workspace_bytes", "ttt_linear_chunked_conv",
+    "ttt_linear_fullbatch_bwd_workspace_bytes", "ttt_linear_fullbatch_bwd",
 }
 
 
@@ -167,3 +168,22 @@ def test_chunked_conv_rejects_bad_arguments(L):
     assert f(*a) == 3
     need = L.ttt_linear_chunked_conv_workspace_bytes(2, 3, 80, 80, 64, 64, 0, 1)
     assert need >= 2 * 2 * 3 * 6400 * 64 * 2
+
+
+def test_backward_rejects_bad_arguments(L):
+    f = L.ttt_linear_fullbatch_bwd
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1, 128, 64, 1.0, 1, FAKE, 1 << 30, None]
+    for idx in (4, 5, 8):  # dout, dq, dw0
+        a = list(ok)
+        a[idx] = None
+        assert f(*a) == 1
+    a = list(ok)
+    a[6] = MISALIGNED
+    assert f(*a) == 1
+    a = list(ok)
+    a[12] = 256
+    assert f(*a) == 2
+    a = list(ok)
+    a[16] = 64
+    assert f(*a) == 3
+    assert L.ttt_linear_fullbatch_bwd_workspace_bytes(2, 1, 128, 48, 0) >= 2 * 6 * 48 * 48 * 4
