@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, cpu baseline, other paths")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--only", choices=["dwconv", "mlp", "chunked"], default=None,
+    ap.add_argument("--only", choices=["dwconv", "mlp", "chunked", "backward", "oneway", "minibatch", "convscan"],
+                    default=None,
                     help="time one other path alone (used for per-kernel ncu captures)")
     return ap.parse_args()
 
@@ -544,6 +545,58 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=
                                     "us_per_chunk_step": ms * 1e3 / 100,
                                     "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9,
                                     "l2": f"{R} rotating sets of {nb / 1e6:.1f} MB (> 4x L2)"}
+        del S, ws
+    if only in (None, "backward"):  # TTT-Linear backward at the forward's shape, B=32, 56x56, d=64
+        nb = 7 * 32 * 3136 * 64 * 2  # read Q, K, V, dO; write dQ, dK, dV
+        R = sets_for(nb)
+
+        def mk(r):
+            x = inputs.linear_bwd_inputs(32, 1, 3136, 64, seed=400 + r)
+            return {"q": x["q"], "k": x["k"], "v": x["v"], "w0": x["w0"], "dout": x["dout"]}
+        S = rotating(mk, R)
+        for x in S:
+            x["dk"], x["dv"], x["dw0"] = torch.empty_like(x["q"]), torch.empty_like(x["q"]), torch.empty_like(x["w0"])
+        ws = workspace(ttt.ttt_linear_fullbatch_bwd_workspace_bytes(32, 1, 3136, 64, 1))
+        ms = timed(lambda i: ttt.ttt_linear_fullbatch_bwd(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"], S[i]["dout"],
+                                                          S[i]["out"], S[i]["dk"], S[i]["dv"], S[i]["dw0"], 1.0, ws,
+                                                          stream), R, 200)
+        res["linear_bwd_56x56_d64"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
+                                       "hbm_gbs": nb / (ms / 1e3) / 1e9,
+                                       "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / hbm_peak,
+                                       "bytes": "read Q, K, V, dO and write dQ, dK, dV once (the kernels "
+                                                "read dO, K, V twice)", "kernels_per_call": 4,
+                                       "l2": f"{R} rotating sets of {nb / 1e6:.1f} MB (> 4x L2)"}
+        del S, ws
+    if only in (None, "oneway"):  # one-way (raster) chunked scan, 80x80, chunk 64
+        nb = 8 * 8 * 3 * 6400 * 64
+        R = sets_for(nb)
+        S = rotating(lambda r: inputs.chunked_inputs(8, 3, 6400, 64, seed=500 + r), R)
+        ms = timed(lambda i: ttt.ttt_linear_chunked(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"], S[i]["out"], 64,
+                                                    1.0, 1, None, stream), R, 50)
+        res["chunked_one_way_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
+                                            "us_per_chunk_step": ms * 1e3 / 100,
+                                            "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9}
+        del S
+    if only in (None, "convscan"):  # Conv2d-preprocessed bidirectional scan, 80x80, chunk 64
+        nb = 8 * 8 * 3 * 6400 * 64
+        R = sets_for(nb)
+        S = rotating(lambda r: inputs.chunked_conv_inputs(8, 3, 80, 80, 64, seed=600 + r), R)
+        ws = workspace(ttt.ttt_linear_chunked_conv_workspace_bytes(8, 3, 80, 80, 64, 64, 0, 1))
+        ms = timed(lambda i: ttt.ttt_linear_chunked_conv(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"], S[i]["wk"],
+                                                         S[i]["wv"], S[i]["out"], 80, 80, 64, 1.0, 0, ws, stream), R, 50)
+        res["chunked_conv_80x80_b64"] = {"ms": ms, "tokens_per_s": 8 * 6400 / (ms / 1e3),
+                                         "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9, "kernels_per_call": 3}
+        del S, ws
+    if only in (None, "minibatch"):  # mini-batch training, chunks of 64, 2 epochs, B=32, 56x56
+        nb = 8 * 32 * 3136 * 64
+        R = sets_for(nb)
+        S = rotating(lambda r: inputs.linear_inputs(32, 1, 3136, 64, seed=700 + r), R)
+        ws = workspace(ttt.ttt_linear_minibatch_workspace_bytes(32, 1, 3136, 64, 64, 2, 1))
+        ms = timed(lambda i: ttt.ttt_linear_minibatch(S[i]["q"], S[i]["k"], S[i]["v"], S[i]["w0"], S[i]["out"], 64,
+                                                      2, None, 1.0, ws, stream), R, 5)
+        res["minibatch_56x56_b64_e2"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
+                                         "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9, "kernels_per_call": 2,
+                                         "note": "CUDA-core kernels (one block per unit scans the chunks)"}
         del S, ws
     assert ttt.device_error() == 0
     return res

@@ -473,4 +473,47 @@ __global__ void __launch_bounds__(TPB) dwconv_prep(const T* __restrict__ x, cons
     y[u * N * d + e] = from_f<T>(acc);
 }
 
+// bf16 version for d % 8 == 0: one thread makes 8 consecutive features of one token (16-byte
+// loads of the 3x3 neighbourhood, the head's filters staged in shared memory); blockIdx.z picks
+// K (0) or V (1), so one launch preprocesses both.
+__global__ void __launch_bounds__(TPB) dwconv_prep2_bf16(const __nv_bfloat16* __restrict__ k,
+                                                         const __nv_bfloat16* __restrict__ v,
+                                                         const float* __restrict__ wk, const float* __restrict__ wv,
+                                                         __nv_bfloat16* __restrict__ kp, __nv_bfloat16* __restrict__ vp,
+                                                         int H, int Hg, int Wg, int d) {
+    extern __shared__ float wsm[];  // [d][9]
+    const long long u = blockIdx.x;
+    const bool isv = blockIdx.z != 0;
+    const float* w = (isv ? wv : wk) + (u % H) * d * 9;
+    for (int e = threadIdx.x; e < d * 9; e += TPB) wsm[e] = w[e];
+    __syncthreads();
+    const long long N = (long long)Hg * Wg;
+    const int g8 = d / 8;
+    const long long e = (long long)blockIdx.y * TPB + threadIdx.x;  // (token, 8-feature group)
+    if (e >= N * g8) return;
+    const long long t = e / g8;
+    const int f0 = (int)(e % g8) * 8;
+    const int py = (int)(t / Wg), px = (int)(t % Wg);
+    const __nv_bfloat16* xu = (isv ? v : k) + u * N * d;
+    float acc[8] = {};
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            const int yy = py + a - 1, xx = px + b - 1;
+            if (yy < 0 || yy >= Hg || xx < 0 || xx >= Wg) continue;
+            const uint4 raw = *reinterpret_cast<const uint4*>(xu + ((long long)yy * Wg + xx) * d + f0);
+            const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(pr[i]);
+                acc[2 * i] = fmaf(wsm[(f0 + 2 * i) * 9 + a * 3 + b], f.x, acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wsm[(f0 + 2 * i + 1) * 9 + a * 3 + b], f.y, acc[2 * i + 1]);
+            }
+        }
+    *reinterpret_cast<uint4*>((isv ? vp : kp) + u * N * d + t * d + f0) =
+        make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
+                   pack_bf16(acc[6], acc[7]));
+}
+
 }  // namespace simt

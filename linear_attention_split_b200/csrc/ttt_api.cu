@@ -969,7 +969,16 @@ int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const f
     void* vp = w + align256((size_t)U * N * d * es);
     void* rest = w + 2 * align256((size_t)U * N * d * es);
     const size_t rest_bytes = workspace_bytes - 2 * align256((size_t)U * N * d * es);
-    if (dtype == TTT_BF16) {
+    int prep_launches = 2;
+    if (dtype == TTT_BF16 && d % 8 == 0) {
+        using T = __nv_bfloat16;
+        dim3 grid = grid_units(U, N * (d / 8));
+        grid.z = 2;
+        simt::dwconv_prep2_bf16<<<grid, simt::TPB, d * 9 * 4, st>>>(static_cast<const T*>(k), static_cast<const T*>(v),
+                                                                    wk, wv, static_cast<T*>(kp), static_cast<T*>(vp),
+                                                                    H, Hg, Wg, d);
+        prep_launches = 1;
+    } else if (dtype == TTT_BF16) {
         using T = __nv_bfloat16;
         simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(k), wk,
                                                                          static_cast<T*>(kp), H, Hg, Wg, d);
@@ -982,7 +991,7 @@ int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const f
         simt::dwconv_prep<T><<<grid_units(U, N * d), simt::TPB, 0, st>>>(static_cast<const T*>(v), wv,
                                                                          static_cast<T*>(vp), H, Hg, Wg, d);
     }
-    if (int rc = launched(2)) return rc;
+    if (int rc = launched(prep_launches)) return rc;
     return ttt_linear_chunked(q, kp, vp, w0, out, B, H, (int)N, d, chunk, eta, direction, dtype, rest, rest_bytes,
                               stream);
 }

@@ -91,6 +91,26 @@ def chunked_conv_inputs(B, H, Hg, Wg, d, dtype="bf16", seed=0):
     return inp
 
 
+def block_inputs(B, Hg, Wg, C, H, dtype="bf16", seed=0):
+    """Inputs of the ViT^3 TTT block: x [B, Hg*Wg, C] ~ N(0,1) and the weights, drawn in the
+    order x, Wqkvg, W0, wc, Wo: Wqkvg [C, 4C] (Q, K, V columns ~ N(0, 1/(C d)) so that Q, K, V
+    have the spread N(0,1)/sqrt(d) of the layer's other workloads, gate columns ~ N(0, 1/C)),
+    W0 [H, d, d] fp32 ~ N(0, 1/d), wc [C, 3, 3] fp32 ~ N(0, 1/9), Wo [2C, C] ~ N(0, 1/(2C));
+    x and the two projection matrices are stored in `dtype`."""
+    d = C // H
+    g = _gen(seed)
+    dt = DTYPES[dtype]
+    x = _randn((B, Hg * Wg, C), g, 1.0, dt)
+    w = torch.randn((C, 4 * C), generator=g, dtype=torch.float32)
+    w[:, :3 * C] *= 1.0 / math.sqrt(C * d)
+    w[:, 3 * C:] *= 1.0 / math.sqrt(C)
+    wqkvg = w.to(dt).contiguous()
+    w0 = _randn((H, d, d), g, 1.0 / math.sqrt(d), torch.float32)
+    wc = _randn((C, 3, 3), g, 1.0 / 3.0, torch.float32)
+    wo = _randn((2 * C, C), g, 1.0 / math.sqrt(2 * C), dt)
+    return {"x": x, "wqkvg": wqkvg, "w0": w0, "wc": wc, "wo": wo}
+
+
 # The workloads of the layer, by name.  Each entry: (kind, kwargs for the generator, eta, extra)
 CONFIGS = {
     # TTT-Linear, fp32, one 14x14 grid, one head of d = 64

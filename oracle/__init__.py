@@ -51,6 +51,8 @@ def lib():
         _lib.ttt_oracle_linear_minibatch.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, d, i]
         _lib.ttt_oracle_dwconv_prep.restype = None
         _lib.ttt_oracle_dwconv_prep.argtypes = [p, p, p, i, i, i, i, i]
+        _lib.ttt_oracle_vit3_block.restype = i
+        _lib.ttt_oracle_vit3_block.argtypes = [p, p, p, p, p, p, i, i, i, i, i, d, i]
         _lib.ttt_oracle_linear_chunked_prep.restype = i
         _lib.ttt_oracle_linear_chunked_prep.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, d, i, i]
     return _lib
@@ -239,3 +241,18 @@ def linear_chunked_prep(q, k, v, w0, wk, wv, Hg, Wg, chunk, eta=1.0, direction=0
     if rc != 0:
         raise ValueError("oracle: bad arguments")
     return out
+
+
+# ---------------------------------------------------------------- the ViT^3 block -------
+def vit3_block(x, wqkvg, w0, wc, wo, Hg, Wg, H, eta=1.0, threads=None):
+    """x [B, Hg*Wg, C] -> y [B, Hg*Wg, C] (projections, TTT-Linear core per head, GLU gate,
+    3x3 depthwise-conv branch on x, concat, output projection)."""
+    x, wqkvg, w0, wc, wo = _f64(x), _f64(wqkvg), _f64(w0), _f64(wc), _f64(wo)
+    B, N, C = x.shape
+    assert N == Hg * Wg
+    y = np.empty_like(x)
+    rc = lib().ttt_oracle_vit3_block(_p(x), _p(wqkvg), _p(w0), _p(wc), _p(wo), _p(y), B, Hg, Wg, C, H,
+                                     float(eta), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return y

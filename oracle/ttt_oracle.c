@@ -731,3 +731,91 @@ int ttt_oracle_linear_chunked_prep(const double* q, const double* k, const doubl
     run_units((long)B * H, threads, chunked_prep_unit, &c);
     return 0;
 }
+
+/* ==================================================================================== */
+/* The ViT^3 TTT block around the core (ViT^3 blog, "从官方代码看…": a GLU-style main      */
+/* branch and a 3x3 depthwise-conv branch, concatenated and projected back to the input  */
+/* width; "TTT Block 长什么样": project the input to Q, K, V, train the inner model on     */
+/* (K, V), apply it to Q).  Reading (the pages give no formulas), per image, x [N, C]:    */
+/*   [Q | K | V | G] = x Wqkvg              (Wqkvg [C, 4C]; Q, K, V split into H heads)  */
+/*   O_h = TTT-Linear full-batch step of head h on (Q_h, K_h, V_h) from W0[h]             */
+/*   M = O * sigmoid(G)                     (GLU: a gate from the same input)             */
+/*   D = 3x3 depthwise conv of x on the Hg x Wg grid (taps wc [C, 3, 3], zero padding)    */
+/*   y = [M | D] Wo                         (Wo [2C, C])                                  */
+/* ==================================================================================== */
+
+typedef struct {
+    const double *x, *wqkvg, *w0, *wc, *wo;
+    double* y;
+    int Hg, Wg, C, H;
+    double eta;
+} block_ctx;
+
+static void block_unit(const void* vctx, long b) {
+    const block_ctx* c = (const block_ctx*)vctx;
+    const int C = c->C, H = c->H, d = C / H, N = c->Hg * c->Wg;
+    const double* x = c->x + b * (long)N * C;
+    double* p = (double*)malloc(sizeof(double) * (size_t)N * 4 * C);
+    double* qh = (double*)malloc(sizeof(double) * (size_t)N * d);
+    double* kh = (double*)malloc(sizeof(double) * (size_t)N * d);
+    double* vh = (double*)malloc(sizeof(double) * (size_t)N * d);
+    double* oh = (double*)malloc(sizeof(double) * (size_t)N * d);
+    double* o = (double*)malloc(sizeof(double) * (size_t)N * C);
+    double* z = (double*)malloc(sizeof(double) * (size_t)2 * C);
+    double* gw = (double*)malloc(sizeof(double) * (size_t)d * d);
+    double* ws = (double*)malloc(sizeof(double) * (size_t)d * d);
+    /* projections, token by token */
+    for (int t = 0; t < N; ++t)
+        for (int j = 0; j < 4 * C; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < C; ++i) s += x[(long)t * C + i] * c->wqkvg[(long)i * 4 * C + j];
+            p[(long)t * 4 * C + j] = s;
+        }
+    /* the TTT core per head */
+    for (int h = 0; h < H; ++h) {
+        for (int t = 0; t < N; ++t)
+            for (int e = 0; e < d; ++e) {
+                qh[(long)t * d + e] = p[(long)t * 4 * C + 0 * C + h * d + e];
+                kh[(long)t * d + e] = p[(long)t * 4 * C + 1 * C + h * d + e];
+                vh[(long)t * d + e] = p[(long)t * 4 * C + 2 * C + h * d + e];
+            }
+        const double* w0 = c->w0 + (long)h * d * d;
+        ttt_oracle_linear_grad(kh, vh, w0, N, d, gw);
+        for (long e = 0; e < (long)d * d; ++e) ws[e] = w0[e] - c->eta * gw[e];
+        linear_apply(qh, ws, N, d, oh);
+        for (int t = 0; t < N; ++t)
+            for (int e = 0; e < d; ++e) o[(long)t * C + h * d + e] = oh[(long)t * d + e];
+    }
+    /* gate, conv branch, concat, output projection, token by token */
+    for (int t = 0; t < N; ++t) {
+        const int py = t / c->Wg, px = t % c->Wg;
+        for (int ch = 0; ch < C; ++ch) {
+            const double g = p[(long)t * 4 * C + 3 * C + ch];
+            z[ch] = o[(long)t * C + ch] / (1.0 + exp(-g));
+            z[C + ch] = dwconv_at(x, c->wc + ch * 9, c->Hg, c->Wg, C, py, px, ch);
+        }
+        for (int j = 0; j < C; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < 2 * C; ++i) s += z[i] * c->wo[(long)i * C + j];
+            c->y[(b * (long)N + t) * C + j] = s;
+        }
+    }
+    free(p);
+    free(qh);
+    free(kh);
+    free(vh);
+    free(oh);
+    free(o);
+    free(z);
+    free(gw);
+    free(ws);
+}
+
+int ttt_oracle_vit3_block(const double* x, const double* wqkvg, const double* w0, const double* wc,
+                          const double* wo, double* y, int B, int Hg, int Wg, int C, int H, double eta,
+                          int threads) {
+    if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0 || H <= 0 || C % H != 0) return 1;
+    block_ctx c = {x, wqkvg, w0, wc, wo, y, Hg, Wg, C, H, eta};
+    run_units((long)B, threads, block_unit, &c);
+    return 0;
+}

@@ -67,6 +67,12 @@ int ttt_oracle_linear_chunked_prep(const double* q, const double* k, const doubl
                                    double* out, int B, int H, int Hg, int Wg, int d, int chunk,
                                    double eta, int direction, int threads);
 
+/* ViT^3 TTT block: x [B, Hg*Wg, C] -> y [B, Hg*Wg, C]; wqkvg [C, 4C], w0 [H, C/H, C/H],
+ * wc [C, 3, 3], wo [2C, C] */
+int ttt_oracle_vit3_block(const double* x, const double* wqkvg, const double* w0, const double* wc,
+                          const double* wo, double* y, int B, int Hg, int Wg, int C, int H, double eta,
+                          int threads);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,5 +1,5 @@
-"""Pins of the oracle's backward, mini-batch / multi-epoch and conv-preprocessing functions
-(CPU only).  Each is tied to something other than itself: hand-worked fixtures
+"""Pins of the oracle's backward, mini-batch / multi-epoch, conv-preprocessing and ViT^3 block
+functions (CPU only).  Each is tied to something other than itself: hand-worked fixtures
 (tests/golden), finite differences of the pinned forward oracle, torch autograd of a
 re-statement built from library matmuls, closed forms of the linear model's affine updates,
 special cases, and torch's conv2d."""
@@ -12,6 +12,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle
+from linear_attention_split_b200 import inputs
 
 RNG = np.random.default_rng(1234)
 
@@ -205,3 +206,57 @@ def test_chunked_unidirectional_sums_to_bidirectional():
     r = oracle.linear_chunked(q, k, v, w0, 8, direction=-1)
     both = oracle.linear_chunked(q, k, v, w0, 8, direction=0)
     np.testing.assert_allclose(f + r, both, rtol=1e-12, atol=1e-13)
+
+
+# ====================================================================== the ViT^3 block ==
+def torch_block(x, wqkvg, w0, wc, wo, Hg, Wg, H, eta):
+    """The block composed from library operators (matmul, conv2d, sigmoid) around the
+    pinned TTT-Linear core of the oracle."""
+    B, N, C = x.shape
+    d = C // H
+    xt = torch.tensor(x)
+    p = xt @ torch.tensor(wqkvg)
+    q, k, v, g = p[..., :C], p[..., C:2 * C], p[..., 2 * C:3 * C], p[..., 3 * C:]
+    split = lambda t: t.reshape(B, N, H, d).permute(0, 2, 1, 3).numpy()
+    o, _ = oracle.linear_fullbatch(split(q), split(k), split(v), w0, eta=eta)
+    o = torch.tensor(o).permute(0, 2, 1, 3).reshape(B, N, C)
+    m = o * torch.sigmoid(g)
+    xi = xt.reshape(B, Hg, Wg, C).permute(0, 3, 1, 2)
+    dc = F.conv2d(xi, torch.tensor(wc).reshape(C, 1, 3, 3), padding=1, groups=C)
+    dc = dc.permute(0, 2, 3, 1).reshape(B, N, C)
+    return (torch.cat([m, dc], dim=-1) @ torch.tensor(wo)).numpy()
+
+
+def test_block_is_composition_of_library_operators():
+    B, Hg, Wg, C, H = 2, 5, 6, 8, 2
+    inp = {k: v.double().numpy() for k, v in inputs.block_inputs(B, Hg, Wg, C, H, dtype="f32", seed=3).items()}
+    for eta in (1.0, 0.4):
+        got = oracle.vit3_block(inp["x"], inp["wqkvg"], inp["w0"], inp["wc"], inp["wo"], Hg, Wg, H, eta=eta)
+        ref = torch_block(inp["x"], inp["wqkvg"], inp["w0"], inp["wc"], inp["wo"], Hg, Wg, H, eta)
+        np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_block_special_cases():
+    """Zero gate columns give sigmoid(0) = 1/2 exactly; a Wo that keeps only the conv half
+    leaves the 3x3 depthwise conv of x (torch conv2d) times that half."""
+    B, Hg, Wg, C, H = 1, 4, 4, 4, 1
+    x = rnd(B, Hg * Wg, C)
+    wqkvg = rnd(C, 4 * C, scale=0.3)
+    w0 = rnd(H, C, C, scale=0.5)
+    wc = rnd(C, 3, 3)
+    wo = np.zeros((2 * C, C))
+    wo[C:, :] = np.eye(C)
+    y = oracle.vit3_block(x, wqkvg, w0, wc, wo, Hg, Wg, H)
+    xi = torch.tensor(x).reshape(B, Hg, Wg, C).permute(0, 3, 1, 2)
+    dc = F.conv2d(xi, torch.tensor(wc).reshape(C, 1, 3, 3), padding=1, groups=C)
+    np.testing.assert_allclose(y, dc.permute(0, 2, 3, 1).reshape(B, Hg * Wg, C).numpy(), rtol=1e-12, atol=1e-13)
+    wq = wqkvg.copy()
+    wq[:, 3 * C:] = 0.0
+    wo2 = np.zeros((2 * C, C))
+    wo2[:C, :] = np.eye(C)
+    y2 = oracle.vit3_block(x, wq, w0, wc, wo2, Hg, Wg, H)
+    q = x @ wq[:, :C]
+    k = x @ wq[:, C:2 * C]
+    v = x @ wq[:, 2 * C:3 * C]
+    o, _ = oracle.linear_fullbatch(q[:, None], k[:, None], v[:, None], w0)
+    np.testing.assert_allclose(y2, 0.5 * o[:, 0], rtol=1e-12, atol=1e-13)
