@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, cpu baseline, other paths")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--only", choices=["dwconv", "mlp", "chunked", "backward", "oneway", "minibatch", "convscan"],
+    ap.add_argument("--only", choices=["dwconv", "mlp", "chunked", "backward", "oneway", "minibatch", "convscan",
+                                       "block"],
                     default=None,
                     help="time one other path alone (used for per-kernel ncu captures)")
     return ap.parse_args()
@@ -597,6 +598,25 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=
         res["minibatch_56x56_b64_e2"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
                                          "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9, "kernels_per_call": 2,
                                          "note": "CUDA-core kernels (one block per unit scans the chunks)"}
+        del S, ws
+    if only in (None, "block"):  # the ViT^3 block at the stage-1 width: B=32, 56x56, C=64, 2 heads of 32
+        nb = 32 * 3136 * 64 * 2 * 2  # x in, y out
+        R = sets_for(nb * 4)
+
+        def mk(r):
+            x = inputs.block_inputs(32, 56, 56, 64, 2, seed=800 + r)
+            x["q"] = x["x"]  # rotating() sizes "out" after "q"
+            return x
+        S = rotating(mk, R)
+        ws = workspace(ttt.ttt_vit3_block_workspace_bytes(32, 56, 56, 64, 2, 1))
+        ms = timed(lambda i: ttt.ttt_vit3_block(S[i]["x"], S[i]["wqkvg"], S[i]["w0"], S[i]["wc"], S[i]["wo"],
+                                                S[i]["out"], 56, 56, 2, 1.0, ws, stream), R, 100)
+        inter = 32 * 3136 * 64 * 2 * (1 + 5 + 3 + 1 + 1 + 1)  # x, QKVG+O writes, QKV+O+G reads, x again, y
+        res["vit3_block_56x56_c64_h2"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
+                                          "hbm_gbs_in_out": nb / (ms / 1e3) / 1e9,
+                                          "hbm_gbs_with_intermediates": inter / (ms / 1e3) / 1e9,
+                                          "frac_of_hbm_peak_with_intermediates": inter / (ms / 1e3) / 1e9 / hbm_peak,
+                                          "kernels_per_call": 3}
         del S, ws
     assert ttt.device_error() == 0
     return res

@@ -95,6 +95,26 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* --------------------------------------------------------------------------------------
+ * The ViT^3 TTT block around the TTT-Linear core (ViT^3 blog: the block projects its input to
+ * Q, K, V, trains the inner model on (K, V) and applies it to Q -- "TTT Block 长什么样"; the
+ * official code joins a GLU-style main branch and a 3x3 depthwise-conv branch, concatenates
+ * them and projects back to the input width -- "从官方代码看…").  This library's reading,
+ * per image with x [N, C] on the Hg x Wg grid (token index row*Wg + col):
+ *     [Q | K | V | G] = x Wqkvg              (Q, K, V split into H heads of d = C/H)
+ *     O = ttt_linear_fullbatch(Q, K, V, W0)  (per head, learning rate eta)
+ *     y = [O * sigmoid(G) | dwconv3x3(x)] Wo  (taps wc, zero padding, no bias)
+ *   x, y  : [B, Hg*Wg, C] dtype;   wqkvg : [C, 4C] dtype;   wo : [2C, C] dtype
+ *   w0    : [H, d, d] fp32;        wc    : [C, 3, 3] fp32
+ * bf16 with C = 64 and d in {32, 64} runs the tensor-core kernels; everything else the
+ * CUDA-core kernels.  The workspace (always needed) holds Q, K, V, G and O.  Errors as for
+ * the other entry points (C % H != 0 is TTT_ERR_INVALID_ARG).
+ * ------------------------------------------------------------------------------------ */
+size_t ttt_vit3_block_workspace_bytes(int B, int Hg, int Wg, int C, int H, int dtype);
+int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const float* wc, const void* wo, void* y,
+                   int B, int Hg, int Wg, int C, int H, float eta, int dtype, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------
  * Backward of the TTT-Linear full-batch step (outer training through the inner step: the
  * ViT^3 abstract's "parallelizable computation"; the ViT^3 blog notes the official code writes
  * the closed-form gradient of the inner step by hand).  For an upstream gradient dO = dL/dO of

@@ -1,0 +1,256 @@
+// block_tc.cuh -- the ViT^3 TTT block around the TTT-Linear core on the tcgen05 tensor cores,
+// bf16, block width C = 64 (the high-resolution stage-1 width of the hierarchical model).
+//
+// Operation (ViT^3 blog: the block projects its input to Q, K, V, trains the inner model on
+// (K, V) and applies it to Q -- "TTT Block 长什么样" -- and its official code joins a GLU-style
+// main branch with a 3x3 depthwise-conv branch, concatenates them and projects back to the
+// input width -- "从官方代码看…"), per image with x [N, C] on the Hg x Wg grid:
+//     [Q | K | V | G] = x Wqkvg,   O = TTT-Linear(Q, K, V) per head,
+//     y = [O * sigmoid(G) | dwconv3x3(x)] Wo
+// Two kernels around the core (the full-batch step needs every token's K and V before any
+// output, so the core is a kernel of its own):
+//   proj : per 128-token tile, x (TMA) times Wqkvg (resident, MN-major) into 256 TMEM columns;
+//          the epilogue writes Q, K, V head-split [B, H, N, d] and G [B, N, C] in bf16.
+//   out  : per 128-token tile, four warps build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128,
+//          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows,
+//          the conv from the 3x3 neighbourhood of x (16-byte loads, fp32 taps) -- then one MMA
+//          chain Z_hi Wo + Z_lo Wo (K = 128, N = 64) and the epilogue stores y in bf16.
+// No token-tile output is written twice and no intermediate of the out kernel (Z) goes to HBM.
+#pragma once
+#include "common.cuh"
+
+namespace blk {
+
+constexpr int C = 64;
+constexpr int ROWB = C * 2;             // 128 bytes per token row
+constexpr int MT = 128;                 // tokens per tile
+constexpr int XT = MT * ROWB;           // 16 KB
+constexpr int WQ = C * 4 * C * 2;       // Wqkvg, 32 KB (four 64-column atoms)
+constexpr int ZT = MT * 2 * C * 2;      // Z hi or lo, 32 KB each (two 64-column K-major atoms)
+constexpr int WO = 2 * C * C * 2;       // Wo, 16 KB
+constexpr int THREADS = 160;            // four row warps (epilogue) + one issuer warp
+
+struct PParams {
+    __nv_bfloat16 *q, *k, *v, *g;       // [B, H, N, d] x 3, [B, N, C]
+    long long rows;                     // B * N
+    int N, H, d;
+};
+struct PBars {
+    uint64_t full, done;
+    uint32_t tmem_base;
+};
+constexpr int p_smem_bytes() { return XT + WQ + (int)sizeof(PBars) + 1024; }
+
+__global__ void __launch_bounds__(THREADS, 1)
+    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const PParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ws = xs + XT;
+    PBars* bars = reinterpret_cast<PBars*>(ws + WQ);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row0 = (long long)blockIdx.x * MT;
+    if (threadIdx.x == 128) {
+        mbar_init(&bars->full, 1);
+        mbar_init(&bars->done, 1);
+        mbar_fence_init();
+    }
+    if (warp == 4) tc::alloc(&bars->tmem_base, 256);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    if (warp == 4) {
+        if (lane == 0) {
+            mbar_expect_tx(&bars->full, XT + WQ);  // out-of-range rows are zero-filled and counted
+            tma_load_3d(xs, &tm_x, 0, (int)row0, 0, &bars->full);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) tma_load_3d(ws + a * 8192, &tm_w, a * 64, 0, 0, &bars->full);
+            mbar_wait(&bars->full, 0, TTT_DEVERR_TIMEOUT_TMA);
+            tc::fence_after();
+            const uint32_t xa = smem_u32(xs), wa = smem_u32(ws);
+            constexpr uint32_t ID = tc::idesc_bf16(128, 256, 0, 1);  // A K-major, B MN-major, N = 256
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16(tmem, tc::smem_desc(xa + ks * 32, 16, 1024, 2), tc::smem_desc(wa + ks * 2048, 8192, 1024, 2),
+                             ID, ks > 0 ? 1 : 0);
+            tc::commit(&bars->done);
+        }
+    } else {
+        const int row = warp * 32 + lane;
+        const long long R = row0 + row;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
+        tc::fence_after();
+        const long long b = R / p.N, t = R % p.N;
+#pragma unroll 1
+        for (int j0 = 0; j0 < 4 * C; j0 += 16) {
+            float v[16];
+            tc::ld16(lane_base + j0, v);
+            tc::wait_ld();
+            if (R >= p.rows) continue;
+            const int which = j0 / C, c = j0 % C;
+            __nv_bfloat16* dst;
+            if (which == 3) {
+                dst = p.g + R * C + c;
+            } else {
+                const int h = c / p.d, e = c % p.d;
+                __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : p.v;
+                dst = base + ((b * p.H + h) * p.N + t) * p.d + e;
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            d4[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            d4[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                               pack_bf16(v[14], v[15]));
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 4) tc::dealloc(tmem, 256);
+}
+
+struct OParams {
+    const __nv_bfloat16* x;             // [B, N, C]
+    const __nv_bfloat16* o;             // [B, H, N, d] (the core's output)
+    const __nv_bfloat16* g;             // [B, N, C]
+    const float* wc;                    // [C, 3, 3]
+    __nv_bfloat16* y;                   // [B, N, C]
+    long long rows;
+    int N, Hg, Wg, H, d;
+};
+struct OBars {
+    uint64_t wfull, zready, done;
+    uint32_t tmem_base;
+};
+constexpr int o_smem_bytes() { return 2 * ZT + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+// eight fp32 values -> bf16 hi and lo = bf16(x - hi), packed
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+        const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h[i]));
+        l[i] = pack_bf16(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    out_kernel(const __grid_constant__ CUtensorMap tm_wo, const OParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* zs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* zl = zs + ZT;                 // Z lo
+    uint8_t* wos = zl + ZT;
+    float* wcs = reinterpret_cast<float*>(wos + WO);
+    OBars* bars = reinterpret_cast<OBars*>(wcs + C * 9);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row0 = (long long)blockIdx.x * MT;
+    if (threadIdx.x == 128) {
+        mbar_init(&bars->wfull, 1);
+        mbar_init(&bars->zready, 4);
+        mbar_init(&bars->done, 1);
+        mbar_fence_init();
+    }
+    for (int e = threadIdx.x; e < C * 9; e += THREADS) wcs[e] = p.wc[e];
+    if (warp == 4) tc::alloc(&bars->tmem_base, 64);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    if (warp == 4) {
+        if (lane == 0) {
+            mbar_expect_tx(&bars->wfull, WO);
+            tma_load_3d(wos, &tm_wo, 0, 0, 0, &bars->wfull);
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+            mbar_wait(&bars->zready, 0, TTT_DEVERR_TIMEOUT_PEER);
+            tc::fence_after();
+            const uint32_t wa = smem_u32(wos);
+            constexpr uint32_t ID = tc::idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl) {
+                const uint32_t za = smem_u32(hl ? zl : zs);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16(tmem, tc::smem_desc(za + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
+                                 tc::smem_desc(wa + ks * 2048, 8192, 1024, 2), ID, (hl > 0 || ks > 0) ? 1 : 0);
+            }
+            tc::commit(&bars->done);
+        }
+    } else {
+        const int row = warp * 32 + lane;
+        const long long R = row0 + row;
+        const bool valid = R < p.rows;
+        const long long b = R / p.N, t = R % p.N;
+        const int py = (int)(t / p.Wg), px = (int)(t % p.Wg);
+        // Z columns 0-63: O * sigmoid(G); columns 64-127: 3x3 depthwise conv of x
+#pragma unroll 1
+        for (int c = 0; c < C; c += 8) {
+            uint4 mz = make_uint4(0, 0, 0, 0), dz = mz, mzl = mz, dzl = mz;
+            if (valid) {
+                const int h = c / p.d, e = c % p.d;
+                const uint4 ov = *reinterpret_cast<const uint4*>(p.o + ((b * p.H + h) * p.N + t) * p.d + e);
+                const uint4 gv = *reinterpret_cast<const uint4*>(p.g + R * C + c);
+                const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+                float m[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 of = __bfloat1622float2(o2[i]), gf = __bfloat1622float2(g2[i]);
+                    m[2 * i] = of.x * sigmoidf_(gf.x);
+                    m[2 * i + 1] = of.y * sigmoidf_(gf.y);
+                }
+                split8(m, mz, mzl);
+                float acc[8] = {};
+                const __nv_bfloat16* xb = p.x + b * p.N * C;
+#pragma unroll
+                for (int a = 0; a < 3; ++a)
+#pragma unroll
+                    for (int bb = 0; bb < 3; ++bb) {
+                        const int yy = py + a - 1, xx = px + bb - 1;
+                        if (yy < 0 || yy >= p.Hg || xx < 0 || xx >= p.Wg) continue;
+                        const uint4 raw = *reinterpret_cast<const uint4*>(xb + ((long long)yy * p.Wg + xx) * C + c);
+                        const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = __bfloat1622float2(r2[i]);
+                            acc[2 * i] = fmaf(wcs[(c + 2 * i) * 9 + a * 3 + bb], f.x, acc[2 * i]);
+                            acc[2 * i + 1] = fmaf(wcs[(c + 2 * i + 1) * 9 + a * 3 + bb], f.y, acc[2 * i + 1]);
+                        }
+                    }
+                split8(acc, dz, dzl);
+            }
+            const uint32_t off = swz<3>((uint32_t)row * ROWB + c * 2);
+            *reinterpret_cast<uint4*>(zs + off) = mz;
+            *reinterpret_cast<uint4*>(zs + 16384 + off) = dz;
+            *reinterpret_cast<uint4*>(zl + off) = mzl;
+            *reinterpret_cast<uint4*>(zl + 16384 + off) = dzl;
+        }
+        fence_proxy_async_smem();  // read next by the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->zready);
+        mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
+        tc::fence_after();
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tc::ld16(lane_base + half * 32, &v[0]);
+            tc::ld16(lane_base + half * 32 + 16, &v[16]);
+            tc::wait_ld();
+            if (valid) {
+                uint4* d4 = reinterpret_cast<uint4*>(p.y + R * C + half * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    d4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                       pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+            }
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 4) tc::dealloc(tmem, 64);
+}
+
+}  // namespace blk

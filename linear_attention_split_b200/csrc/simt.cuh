@@ -446,6 +446,69 @@ __global__ void __launch_bounds__(TPB) linear_bwd_dw0(const float* __restrict__ 
     dw0[(long long)h * dd + e] = s;
 }
 
+// ------------------------------------------------------------------ ViT^3 block ---------
+// [Q | K | V | G] = x Wqkvg at element (row R = b N + t, column j): Q, K, V head-split.
+template <typename T>
+__global__ void __launch_bounds__(TPB) block_proj(const T* __restrict__ x, const T* __restrict__ w, T* __restrict__ q,
+                                                  T* __restrict__ k, T* __restrict__ v, T* __restrict__ g,
+                                                  long long rows, int N, int C, int H) {
+    const long long e = (long long)blockIdx.x * TPB + threadIdx.x;
+    if (e >= rows * 4 * C) return;
+    const long long R = e / (4 * C);
+    const int j = (int)(e % (4 * C));
+    float s = 0.f;
+    for (int i = 0; i < C; ++i) s = fmaf(to_f(x[R * C + i]), to_f(w[(long long)i * 4 * C + j]), s);
+    const int which = j / C, c = j % C, d = C / H;
+    const long long b = R / N, t = R % N;
+    if (which == 3) {
+        g[R * C + c] = from_f<T>(s);
+    } else {
+        T* base = which == 0 ? q : which == 1 ? k : v;
+        base[((b * H + c / d) * N + t) * d + c % d] = from_f<T>(s);
+    }
+}
+
+// Z[R] = [O * sigmoid(G) | dwconv3x3(x)] (fp32) at element (R, j), j < 2C
+template <typename T>
+__global__ void __launch_bounds__(TPB) block_z(const T* __restrict__ x, const T* __restrict__ o,
+                                               const T* __restrict__ g, const float* __restrict__ wc,
+                                               float* __restrict__ z, long long rows, int N, int Hg, int Wg, int C,
+                                               int H) {
+    const long long e = (long long)blockIdx.x * TPB + threadIdx.x;
+    if (e >= rows * 2 * C) return;
+    const long long R = e / (2 * C);
+    const int j = (int)(e % (2 * C));
+    const long long b = R / N, t = R % N;
+    const int d = C / H;
+    if (j < C) {
+        const float gv = to_f(g[R * C + j]);
+        z[e] = to_f(o[((b * H + j / d) * N + t) * d + j % d]) / (1.f + expf(-gv));
+    } else {
+        const int c = j - C, py = (int)(t / Wg), px = (int)(t % Wg);
+        float acc = 0.f;
+        for (int a = 0; a < 3; ++a)
+            for (int bb = 0; bb < 3; ++bb) {
+                const int yy = py + a - 1, xx = px + bb - 1;
+                if (yy >= 0 && yy < Hg && xx >= 0 && xx < Wg)
+                    acc = fmaf(wc[c * 9 + a * 3 + bb], to_f(x[(b * N + (long long)yy * Wg + xx) * C + c]), acc);
+            }
+        z[e] = acc;
+    }
+}
+
+// y = Z Wo at element (R, j)
+template <typename T>
+__global__ void __launch_bounds__(TPB) block_outproj(const float* __restrict__ z, const T* __restrict__ wo,
+                                                     T* __restrict__ y, long long rows, int C) {
+    const long long e = (long long)blockIdx.x * TPB + threadIdx.x;
+    if (e >= rows * C) return;
+    const long long R = e / C;
+    const int j = (int)(e % C);
+    float s = 0.f;
+    for (int i = 0; i < 2 * C; ++i) s = fmaf(z[R * 2 * C + i], to_f(wo[(long long)i * C + j]), s);
+    y[e] = from_f<T>(s);
+}
+
 // ------------------------------------------------------------------ conv preprocessing --
 // x' = 3x3 depthwise conv of x over the Hg x Wg token grid of each unit (zero padding, no
 // bias): one filter per feature of each head, taps w [H][d][3][3]; x, y [U][Hg*Wg][d].

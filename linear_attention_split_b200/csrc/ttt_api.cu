@@ -18,6 +18,7 @@
 #include "linear_tc.cuh"
 #include "linear_tc5.cuh"
 #include "linear_bwd_tc.cuh"
+#include "block_tc.cuh"
 #include "dwconv_fused.cuh"
 #include "chunked_tc.cuh"
 #include "mlp_tc.cuh"
@@ -369,6 +370,10 @@ int linear_bwd_simt(const void* q, const void* k, const void* v, const float* w0
         static_cast<T*>(dk), static_cast<T*>(dv), N, d, eta_over_n);
     simt::linear_bwd_dw0<<<grid_units(H, (long long)d * d), simt::TPB, 0, st>>>(dw0u, dw0, B, H, d);
     return launched(4);
+}
+
+bool block_tc_ok(int C, int H, int dtype) {
+    return dtype == TTT_BF16 && C == blk::C && (C / H == 32 || C / H == 64) && C % H == 0;
 }
 
 int check_common(const void* q, const void* k, const void* v, const void* out, int dtype, float eta) {
@@ -769,6 +774,120 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
         return linear_simt<__nv_bfloat16>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
     }
     return linear_simt<float>(q, k, v, w0, out, w_star, B, H, N, d, eta, workspace, st);
+}
+
+// ------------------------------------------------------------------ the ViT^3 block -----
+size_t ttt_vit3_block_workspace_bytes(int B, int Hg, int Wg, int C, int H, int dtype) {
+    if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0 || H <= 0 || C % H != 0) return 0;
+    const long long N = (long long)Hg * Wg;
+    if (N > 0x7fffffffLL) return 0;
+    const size_t es = dtype == TTT_BF16 ? 2 : 4;
+    const size_t t = align256((size_t)B * N * C * es);
+    const size_t core = ttt_linear_fullbatch_workspace_bytes(B, H, (int)N, C / H, dtype);
+    const size_t z = block_tc_ok(C, H, dtype) ? 0 : align256((size_t)B * N * 2 * C * 4);
+    return 5 * t + core + z;
+}
+
+int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const float* wc, const void* wo, void* y,
+                   int B, int Hg, int Wg, int C, int H, float eta, int dtype, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    if (!x || !wqkvg || !w0 || !wc || !wo || !y) return TTT_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(wqkvg) || !aligned16(w0) || !aligned16(wc) || !aligned16(wo) || !aligned16(y))
+        return TTT_ERR_INVALID_ARG;
+    if (dtype != TTT_F32 && dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (!std::isfinite(eta)) return TTT_ERR_INVALID_ARG;
+    if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0 || H <= 0 || C % H != 0) return TTT_ERR_INVALID_ARG;
+    const long long N = (long long)Hg * Wg;
+    if (N > 0x7fffffffLL || C / H > 128 || C > 1024) return TTT_ERR_UNSUPPORTED;
+    const size_t need = ttt_vit3_block_workspace_bytes(B, Hg, Wg, C, H, dtype);
+    if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * N;
+    const int d = C / H;
+    const size_t es = dtype == TTT_BF16 ? 2 : 4;
+    const size_t t = align256((size_t)rows * C * es);
+    char* w = static_cast<char*>(workspace);
+    void *q = w, *k = w + t, *v = w + 2 * t, *g = w + 3 * t, *o = w + 4 * t;
+    void* core = w + 5 * t;
+    const size_t core_bytes = ttt_linear_fullbatch_workspace_bytes(B, H, (int)N, d, dtype);
+    if (block_tc_ok(C, H, dtype)) {
+        DeviceInfo* dev = nullptr;
+        if (int rc = current_device(&dev)) return rc;
+        if (blk::p_smem_bytes() > dev->smem_optin || blk::o_smem_bytes() > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
+        if ((rows + blk::MT - 1) / blk::MT > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+        const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+        CUtensorMap tx, tw, two;
+        if (!tmap_bf16_3d(&tx, x, blk::C, (int)rows, 1, blk::MT, sw) ||
+            !tmap_bf16_box(&tw, wqkvg, 4 * blk::C, blk::C, 1, 64, 64, sw) ||
+            !tmap_bf16_box(&two, wo, blk::C, 2 * blk::C, 1, 64, 2 * blk::C, sw))
+            return TTT_ERR_CUDA;
+        if (cudaFuncSetAttribute(blk::proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, blk::p_smem_bytes()) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(blk::out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, blk::o_smem_bytes()) !=
+                cudaSuccess)
+            return TTT_ERR_CUDA;
+        const unsigned tiles = (unsigned)((rows + blk::MT - 1) / blk::MT);
+        blk::PParams pp;
+        pp.q = static_cast<__nv_bfloat16*>(q);
+        pp.k = static_cast<__nv_bfloat16*>(k);
+        pp.v = static_cast<__nv_bfloat16*>(v);
+        pp.g = static_cast<__nv_bfloat16*>(g);
+        pp.rows = rows;
+        pp.N = (int)N;
+        pp.H = H;
+        pp.d = d;
+        blk::proj_kernel<<<tiles, blk::THREADS, blk::p_smem_bytes(), st>>>(tx, tw, pp);
+        if (int rc = launched(1)) return rc;
+        if (int rc = ttt_linear_fullbatch(q, k, v, w0, o, nullptr, B, H, (int)N, d, eta, dtype, core, core_bytes, stream))
+            return rc;
+        blk::OParams op;
+        op.x = static_cast<const __nv_bfloat16*>(x);
+        op.o = static_cast<const __nv_bfloat16*>(o);
+        op.g = static_cast<const __nv_bfloat16*>(g);
+        op.wc = wc;
+        op.y = static_cast<__nv_bfloat16*>(y);
+        op.rows = rows;
+        op.N = (int)N;
+        op.Hg = Hg;
+        op.Wg = Wg;
+        op.H = H;
+        op.d = d;
+        blk::out_kernel<<<tiles, blk::THREADS, blk::o_smem_bytes(), st>>>(two, op);
+        return launched(1);
+    }
+    float* z = reinterpret_cast<float*>(static_cast<char*>(core) + core_bytes);
+    auto blocks = [](long long n) { return (unsigned)((n + simt::TPB - 1) / simt::TPB); };
+    if ((rows * 4 * C + simt::TPB - 1) / simt::TPB > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+    if (dtype == TTT_BF16) {
+        using T = __nv_bfloat16;
+        simt::block_proj<T><<<blocks(rows * 4 * C), simt::TPB, 0, st>>>(
+            static_cast<const T*>(x), static_cast<const T*>(wqkvg), static_cast<T*>(q), static_cast<T*>(k),
+            static_cast<T*>(v), static_cast<T*>(g), rows, (int)N, C, H);
+    } else {
+        using T = float;
+        simt::block_proj<T><<<blocks(rows * 4 * C), simt::TPB, 0, st>>>(
+            static_cast<const T*>(x), static_cast<const T*>(wqkvg), static_cast<T*>(q), static_cast<T*>(k),
+            static_cast<T*>(v), static_cast<T*>(g), rows, (int)N, C, H);
+    }
+    if (int rc = launched(1)) return rc;
+    if (int rc = ttt_linear_fullbatch(q, k, v, w0, o, nullptr, B, H, (int)N, d, eta, dtype, core, core_bytes, stream))
+        return rc;
+    if (dtype == TTT_BF16) {
+        using T = __nv_bfloat16;
+        simt::block_z<T><<<blocks(rows * 2 * C), simt::TPB, 0, st>>>(static_cast<const T*>(x), static_cast<const T*>(o),
+                                                                     static_cast<const T*>(g), wc, z, rows, (int)N,
+                                                                     Hg, Wg, C, H);
+        simt::block_outproj<T><<<blocks(rows * C), simt::TPB, 0, st>>>(z, static_cast<const T*>(wo),
+                                                                       static_cast<T*>(y), rows, C);
+    } else {
+        using T = float;
+        simt::block_z<T><<<blocks(rows * 2 * C), simt::TPB, 0, st>>>(static_cast<const T*>(x), static_cast<const T*>(o),
+                                                                     static_cast<const T*>(g), wc, z, rows, (int)N,
+                                                                     Hg, Wg, C, H);
+        simt::block_outproj<T><<<blocks(rows * C), simt::TPB, 0, st>>>(z, static_cast<const T*>(wo),
+                                                                       static_cast<T*>(y), rows, C);
+    }
+    return launched(2);
 }
 
 // ------------------------------------------------------------------ TTT-Linear backward

@@ -59,6 +59,10 @@ def lib():
         L.ttt_linear_fullbatch_workspace_bytes.argtypes = [i, i, i, i, i]
         L.ttt_linear_fullbatch.restype = i
         L.ttt_linear_fullbatch.argtypes = [p, p, p, p, p, p, i, i, i, i, f, i, p, sz, p]
+        L.ttt_vit3_block_workspace_bytes.restype = sz
+        L.ttt_vit3_block_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.ttt_vit3_block.restype = i
+        L.ttt_vit3_block.argtypes = [p, p, p, p, p, p, i, i, i, i, i, f, i, p, sz, p]
         L.ttt_linear_fullbatch_bwd_workspace_bytes.restype = sz
         L.ttt_linear_fullbatch_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
         L.ttt_linear_fullbatch_bwd.restype = i
@@ -165,6 +169,30 @@ def ttt_linear_fullbatch(q, k, v, w0, out, w_star=None, eta=1.0, workspace=None,
                                     d, float(eta), dt, _ptr(ws), nbytes, _stream(stream))
     _check("ttt_linear_fullbatch", rc)
     return out
+
+
+def ttt_vit3_block_workspace_bytes(B, Hg, Wg, C, H, dtype):
+    return lib().ttt_vit3_block_workspace_bytes(B, Hg, Wg, C, H, dtype)
+
+
+def ttt_vit3_block(x, wqkvg, w0, wc, wo, y, Hg, Wg, H, eta=1.0, workspace=None, stream=None):
+    """The ViT^3 TTT block: x, y [B, Hg*Wg, C]; wqkvg [C, 4C] and wo [2C, C] in x's dtype;
+    w0 [H, C/H, C/H] and wc [C, 3, 3] fp32."""
+    dt = _dtype(x, wqkvg, wo, y)
+    _weights(w0, wc)
+    B, N, C = x.shape
+    if N != Hg * Wg:
+        raise ValueError("N must equal Hg * Wg")
+    ws, nbytes = _workspace(ttt_vit3_block_workspace_bytes(B, Hg, Wg, C, H, dt), workspace, x.device)
+    rc = lib().ttt_vit3_block(_ptr(x), _ptr(wqkvg), _ptr(w0), _ptr(wc), _ptr(wo), _ptr(y), B, Hg, Wg, C, H,
+                              float(eta), dt, _ptr(ws), nbytes, _stream(stream))
+    _check("ttt_vit3_block", rc)
+    return y
+
+
+def vit3_block(x, wqkvg, w0, wc, wo, Hg, Wg, H, eta=1.0):
+    y = torch.empty_like(x)
+    return ttt_vit3_block(x, wqkvg, w0, wc, wo, y, Hg, Wg, H, eta)
 
 
 def ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dtype):

@@ -28,6 +28,7 @@ EXPECTED = {
     "ttt_linear_minibatch_workspace_bytes", "ttt_linear_minibatch",
     "ttt_linear_chunked_conv_workspace_bytes", "ttt_linear_chunked_conv",
     "ttt_linear_fullbatch_bwd_workspace_bytes", "ttt_linear_fullbatch_bwd",
+    "ttt_vit3_block_workspace_bytes", "ttt_vit3_block",
 }
 
 
@@ -187,3 +188,18 @@ def test_backward_rejects_bad_arguments(L):
     a[16] = 64
     assert f(*a) == 3
     assert L.ttt_linear_fullbatch_bwd_workspace_bytes(2, 1, 128, 48, 0) >= 2 * 6 * 48 * 48 * 4
+
+
+def test_block_rejects_bad_arguments(L):
+    f = L.ttt_vit3_block
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 8, 64, 2, 1.0, 1, FAKE, 1 << 30, None]
+    a = list(ok)
+    a[10] = 3  # 64 % 3
+    assert f(*a) == 1
+    a = list(ok)
+    a[3] = None  # wc
+    assert f(*a) == 1
+    a = list(ok)
+    a[14] = 64
+    assert f(*a) == 3
+    assert L.ttt_vit3_block_workspace_bytes(2, 8, 8, 64, 2, 1) >= 5 * 2 * 64 * 64 * 2
