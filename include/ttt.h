@@ -105,8 +105,8 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
  *     y = [O * sigmoid(G) | dwconv3x3(x)] Wo  (taps wc, zero padding, no bias)
  *   x, y  : [B, Hg*Wg, C] dtype;   wqkvg : [C, 4C] dtype;   wo : [2C, C] dtype
  *   w0    : [H, d, d] fp32;        wc    : [C, 3, 3] fp32
- * bf16 with C = 64 and d in {32, 64} runs the tensor-core kernels; everything else the
- * CUDA-core kernels.  The workspace (always needed) holds Q, K, V, G and O.  Errors as for
+ * bf16 with C = 64, d in {32, 64} and Wg <= 63 runs the tensor-core kernels; everything else
+ * the CUDA-core kernels.  The workspace (always needed) holds Q, K, V, G and O.  Errors as for
  * the other entry points (C % H != 0 is TTT_ERR_INVALID_ARG).
  * ------------------------------------------------------------------------------------ */
 size_t ttt_vit3_block_workspace_bytes(int B, int Hg, int Wg, int C, int H, int dtype);

@@ -12,9 +12,11 @@
 //   proj : per 128-token tile, x (TMA) times Wqkvg (resident, MN-major) into 256 TMEM columns;
 //          the epilogue writes Q, K, V head-split [B, H, N, d] and G [B, N, C] in bf16.
 //   out  : per 128-token tile, four warps build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128,
-//          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows,
-//          the conv from the 3x3 neighbourhood of x (16-byte loads, fp32 taps) -- then one MMA
-//          chain Z_hi Wo + Z_lo Wo (K = 128, N = 64) and the epilogue stores y in bf16.
+//          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows
+//          (16-byte loads, all issued up front), the conv from a window of x rows that one TMA
+//          box brings in (the tile's rows and one grid row plus one token on each side, at most
+//          256 rows, so Wg <= 63) -- then one MMA chain Z_hi Wo + Z_lo Wo (K = 128, N = 64) and
+//          the epilogue stores y in bf16.
 // No token-tile output is written twice and no intermediate of the out kernel (Z) goes to HBM.
 #pragma once
 #include "common.cuh"
@@ -28,7 +30,12 @@ constexpr int XT = MT * ROWB;           // 16 KB
 constexpr int WQ = C * 4 * C * 2;       // Wqkvg, 32 KB (four 64-column atoms)
 constexpr int ZT = MT * 2 * C * 2;      // Z hi or lo, 32 KB each (two 64-column K-major atoms)
 constexpr int WO = 2 * C * C * 2;       // Wo, 16 KB
-constexpr int THREADS = 160;            // four row warps (epilogue) + one issuer warp
+constexpr int XW = 256;                 // rows of the x window (tile + halo)
+constexpr int MAX_WG = (XW - MT) / 2 - 1;  // widest grid the window covers (63)
+constexpr int P_WARPS = 8;              // proj: eight epilogue warps (row quarter x column half)
+constexpr int THREADS = 32 * P_WARPS + 32;  // + one issuer warp
+constexpr int O_WARPS = 16;             // out: sixteen Z / epilogue warps (row quarter x 16 channels)
+constexpr int O_THREADS = 32 * O_WARPS + 32;
 
 struct PParams {
     __nv_bfloat16 *q, *k, *v, *g;       // [B, H, N, d] x 3, [B, N, C]
@@ -49,17 +56,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     PBars* bars = reinterpret_cast<PBars*>(ws + WQ);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row0 = (long long)blockIdx.x * MT;
-    if (threadIdx.x == 128) {
+    if (threadIdx.x == 32 * P_WARPS) {
         mbar_init(&bars->full, 1);
         mbar_init(&bars->done, 1);
         mbar_fence_init();
     }
-    if (warp == 4) tc::alloc(&bars->tmem_base, 256);
+    if (warp == P_WARPS) tc::alloc(&bars->tmem_base, 256);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars->tmem_base;
-    if (warp == 4) {
+    if (warp == P_WARPS) {
         if (lane == 0) {
             mbar_expect_tx(&bars->full, XT + WQ);  // out-of-range rows are zero-filled and counted
             tma_load_3d(xs, &tm_x, 0, (int)row0, 0, &bars->full);
@@ -76,14 +83,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::commit(&bars->done);
         }
     } else {
-        const int row = warp * 32 + lane;
+        const int q4 = warp & 3, ch = warp >> 2;  // lane quarter, column half (Q, K | V, G)
+        const int row = q4 * 32 + lane;
         const long long R = row0 + row;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
         mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
         tc::fence_after();
         const long long b = R / p.N, t = R % p.N;
 #pragma unroll 1
-        for (int j0 = 0; j0 < 4 * C; j0 += 16) {
+        for (int j0 = ch * 2 * C; j0 < (ch + 1) * 2 * C; j0 += 16) {
             float v[16];
             tc::ld16(lane_base + j0, v);
             tc::wait_ld();
@@ -105,7 +113,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 4) tc::dealloc(tmem, 256);
+    if (warp == P_WARPS) tc::dealloc(tmem, 256);
 }
 
 struct OParams {
@@ -118,12 +126,12 @@ struct OParams {
     int N, Hg, Wg, H, d;
 };
 struct OBars {
-    uint64_t wfull, zready, done;
+    uint64_t wfull, xfull, zready, done;
     uint32_t tmem_base;
 };
-constexpr int o_smem_bytes() { return 2 * ZT + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
+constexpr int o_smem_bytes() { return 2 * ZT + XW * ROWB + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
 
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
 // eight fp32 values -> bf16 hi and lo = bf16(x - hi), packed
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
     uint32_t h[4], l[4];
@@ -137,30 +145,34 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    out_kernel(const __grid_constant__ CUtensorMap tm_wo, const OParams p) {
+__global__ void __launch_bounds__(O_THREADS, 1)
+    out_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_xw, const OParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* zs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* zl = zs + ZT;                 // Z lo
-    uint8_t* wos = zl + ZT;
+    uint8_t* xw = zl + ZT;                 // x rows row0 - (Wg + 1) .. (128-byte swizzle)
+    uint8_t* wos = xw + XW * ROWB;
     float* wcs = reinterpret_cast<float*>(wos + WO);
     OBars* bars = reinterpret_cast<OBars*>(wcs + C * 9);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row0 = (long long)blockIdx.x * MT;
-    if (threadIdx.x == 128) {
+    if (threadIdx.x == 32 * O_WARPS) {
         mbar_init(&bars->wfull, 1);
-        mbar_init(&bars->zready, 4);
+        mbar_init(&bars->xfull, 1);
+        mbar_init(&bars->zready, O_WARPS);
         mbar_init(&bars->done, 1);
         mbar_fence_init();
     }
-    for (int e = threadIdx.x; e < C * 9; e += THREADS) wcs[e] = p.wc[e];
-    if (warp == 4) tc::alloc(&bars->tmem_base, 64);
+    for (int e = threadIdx.x; e < C * 9; e += O_THREADS) wcs[e] = p.wc[e];
+    if (warp == O_WARPS) tc::alloc(&bars->tmem_base, 64);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars->tmem_base;
-    if (warp == 4) {
+    if (warp == O_WARPS) {
         if (lane == 0) {
+            mbar_expect_tx(&bars->xfull, XW * ROWB);  // rows outside the tensor are zero-filled
+            tma_load_3d(xw, &tm_xw, 0, (int)(row0 - (p.Wg + 1)), 0, &bars->xfull);
             mbar_expect_tx(&bars->wfull, WO);
             tma_load_3d(wos, &tm_wo, 0, 0, 0, &bars->wfull);
             mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
@@ -179,21 +191,30 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::commit(&bars->done);
         }
     } else {
-        const int row = warp * 32 + lane;
+        // warp w: token rows of lane quarter w % 4, channels 16 (w / 4) .. + 15 (two 8-channel chunks)
+        const int q4 = warp & 3, cg = warp >> 2;
+        const int row = q4 * 32 + lane;
         const long long R = row0 + row;
         const bool valid = R < p.rows;
         const long long b = R / p.N, t = R % p.N;
         const int py = (int)(t / p.Wg), px = (int)(t % p.Wg);
-        // Z columns 0-63: O * sigmoid(G); columns 64-127: 3x3 depthwise conv of x
-#pragma unroll 1
-        for (int c = 0; c < C; c += 8) {
+        // the gate half's O and G rows: every load issued before any is used
+        uint4 ov[2], gv[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int c = cg * 16 + q * 8, h = c / p.d, e = c % p.d;
+            ov[q] = valid ? *reinterpret_cast<const uint4*>(p.o + ((b * p.H + h) * p.N + t) * p.d + e) : make_uint4(0, 0, 0, 0);
+            gv[q] = valid ? *reinterpret_cast<const uint4*>(p.g + R * C + c) : make_uint4(0, 0, 0, 0);
+        }
+        mbar_wait(&bars->xfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+        const int wrow = row + p.Wg + 1;  // this token's row in the x window
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int c = cg * 16 + q * 8, chunk = c >> 3;
             uint4 mz = make_uint4(0, 0, 0, 0), dz = mz, mzl = mz, dzl = mz;
             if (valid) {
-                const int h = c / p.d, e = c % p.d;
-                const uint4 ov = *reinterpret_cast<const uint4*>(p.o + ((b * p.H + h) * p.N + t) * p.d + e);
-                const uint4 gv = *reinterpret_cast<const uint4*>(p.g + R * C + c);
-                const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+                const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[q]);
+                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[q]);
                 float m[8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -203,14 +224,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 split8(m, mz, mzl);
                 float acc[8] = {};
-                const __nv_bfloat16* xb = p.x + b * p.N * C;
 #pragma unroll
                 for (int a = 0; a < 3; ++a)
 #pragma unroll
                     for (int bb = 0; bb < 3; ++bb) {
                         const int yy = py + a - 1, xx = px + bb - 1;
                         if (yy < 0 || yy >= p.Hg || xx < 0 || xx >= p.Wg) continue;
-                        const uint4 raw = *reinterpret_cast<const uint4*>(xb + ((long long)yy * p.Wg + xx) * C + c);
+                        const int wr = wrow + (a - 1) * p.Wg + (bb - 1);  // same image: inside the window
+                        const uint4 raw = *reinterpret_cast<const uint4*>(xw + wr * ROWB + ((chunk ^ (wr & 7)) << 4));
                         const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -232,25 +253,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) mbar_arrive(&bars->zready);
         mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
         tc::fence_after();
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tc::ld16(lane_base + half * 32, &v[0]);
-            tc::ld16(lane_base + half * 32 + 16, &v[16]);
-            tc::wait_ld();
-            if (valid) {
-                uint4* d4 = reinterpret_cast<uint4*>(p.y + R * C + half * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    d4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                       pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
-            }
+        // y: this warp's 16 output columns of its lane quarter
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        float v[16];
+        tc::ld16(lane_base + cg * 16, v);
+        tc::wait_ld();
+        if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(p.y + R * C + cg * 16);
+            d4[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            d4[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                               pack_bf16(v[14], v[15]));
         }
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 4) tc::dealloc(tmem, 64);
+    if (warp == O_WARPS) tc::dealloc(tmem, 64);
 }
 
 }  // namespace blk

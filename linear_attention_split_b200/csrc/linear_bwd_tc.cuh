@@ -11,10 +11,10 @@
 //   reduce : CTAs split each unit's tokens (as the forward does); per tile of V, K, Q, dO two
 //            tcgen05 MMAs accumulate [V | K]^T K (C^T and G) and [Q | dO]^T dO (M in its first
 //            64 rows) in TMEM; each CTA writes its partial G, C^T, M (fp32) to the workspace.
-//   finish : one block per unit adds the partials in split order (deterministic) and forms, in
-//            fp32 on the CUDA cores, W*, A and dW0_u; it writes the four d x d right-hand
-//            operands of the token pass -- W*, (eta/N) M^T, -(eta/N) A, (eta/N) M -- each as bf16
-//            hi + lo (row-major rows = output columns, i.e. K-major for the MMA).
+//   finish : sixteen blocks per unit (four output rows each) add the partials in split order
+//            (deterministic) and form, in fp32 on the CUDA cores, W*, A and dW0_u; they write the
+//            four d x d right-hand operands of the token pass -- W*, (eta/N) M^T, -(eta/N) A,
+//            (eta/N) M -- each as bf16 hi + lo (row-major rows = output columns, i.e. K-major).
 //   apply  : per tile of dO, K, V: dQ = dO W*, dV = K (eta/N) M^T-operand, dK = K (-eta/N A) +
 //            V (eta/N M), each product taken as hi + lo into one 64-column TMEM accumulator;
 //            the outputs are written as bf16 over the consumed input tiles and stored by TMA.
@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 }
 
 // ----------------------------------------------------------------------------- finish ----
+// Grid (U, 16): block (u, rb) forms rows 4 rb .. 4 rb + 3 of W*, A and dW0_u (one output per
+// thread).  It adds the S partials (split order) of the four G rows and of all of M, takes W0
+// and the four C rows (columns of C^T), and writes its rows of the eight operands.
 struct FParams {
     const float* part;     // [U][S][3][64][64]
     const float* w0;       // [H][64][64]
@@ -163,8 +166,10 @@ struct FParams {
     int H, S;
     float eta_over_n;
 };
-constexpr int FP = D + 1;  // padded row of the shared-memory matrices
-constexpr int f_smem_bytes() { return 5 * D * FP * 4; }
+constexpr int FROWS = 4;                  // output rows per block
+constexpr int FBLOCKS = D / FROWS;        // blocks per unit
+constexpr int FP = D + 1;                 // padded row of the shared-memory matrices
+constexpr int f_smem_bytes() { return (2 * D * FP + 2 * FROWS * FP) * 4; }
 
 __device__ __forceinline__ void put_hilo(__nv_bfloat16* ops, int m, int row, int col, float x) {
     const __nv_bfloat16 hi = __float2bfloat16_rn(x);
@@ -174,70 +179,50 @@ __device__ __forceinline__ void put_hilo(__nv_bfloat16* ops, int m, int row, int
 
 __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
     extern __shared__ float fsm[];
-    float* Gs = fsm;
-    float* Cts = Gs + D * FP;  // C^T
-    float* Ms = Cts + D * FP;
-    float* W0s = Ms + D * FP;
-    float* Xs = W0s + D * FP;  // W0 M^T
-    const int u = blockIdx.x, tid = threadIdx.x;
+    float* Ms = fsm;                  // all of M
+    float* W0s = Ms + D * FP;         // all of W0
+    float* Gr = W0s + D * FP;         // G rows r0 .. r0 + 3
+    float* Cr = Gr + FROWS * FP;      // C rows r0 .. r0 + 3 (C[r][c] = C^T[c][r])
+    const int u = blockIdx.x, r0 = blockIdx.y * FROWS, tid = threadIdx.x;
     const float* W0 = p.w0 + (size_t)(u % p.H) * DD;
+    const float* part = p.part + (size_t)u * p.S * 3 * DD;
     for (int e = tid; e < DD; e += 256) {
-        float g = 0.f, ct = 0.f, m = 0.f;
-        for (int s = 0; s < p.S; ++s) {  // split order
-            const float* b = p.part + ((size_t)u * p.S + s) * 3 * DD;
-            g += b[e];
-            ct += b[DD + e];
-            m += b[2 * DD + e];
+        float m = 0.f;
+        for (int s = 0; s < p.S; ++s) m += part[(size_t)s * 3 * DD + 2 * DD + e];  // split order
+        Ms[(e >> 6) * FP + (e & 63)] = m;
+        W0s[(e >> 6) * FP + (e & 63)] = W0[e];
+    }
+    {
+        const int i = tid >> 6, c = tid & 63;  // 4 rows x 64 columns
+        float g = 0.f, ct = 0.f;
+        for (int s = 0; s < p.S; ++s) {
+            g += part[(size_t)s * 3 * DD + (r0 + i) * D + c];
+            ct += part[(size_t)s * 3 * DD + DD + c * D + r0 + i];  // C^T[c][r]
         }
-        const int r = e >> 6, c = e & 63;
-        Gs[r * FP + c] = g;
-        Cts[r * FP + c] = ct;
-        Ms[r * FP + c] = m;
-        W0s[r * FP + c] = W0[e];
+        Gr[i * FP + c] = g;
+        Cr[i * FP + c] = ct;
     }
     __syncthreads();
-    const int r0 = (tid >> 4) * 4, c0 = (tid & 15) * 4;
-    float gw[4][4] = {}, x[4][4] = {}, gm[4][4] = {};
+    const int i = tid >> 6, c = tid & 63, r = r0 + i;
+    float gw = 0.f, xrc = 0.f, xcr = 0.f, gm = 0.f;
+#pragma unroll 8
     for (int k = 0; k < D; ++k) {
-        float gr[4], wr[4], wc[4], mt[4], mk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            gr[i] = Gs[(r0 + i) * FP + k];
-            wr[i] = W0s[(r0 + i) * FP + k];
-            wc[i] = W0s[k * FP + c0 + i];
-            mt[i] = Ms[(c0 + i) * FP + k];
-            mk[i] = Ms[k * FP + c0 + i];
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                gw[i][j] = fmaf(gr[i], wc[j], gw[i][j]);  // (G W0)[r][c]
-                x[i][j] = fmaf(wr[i], mt[j], x[i][j]);    // (W0 M^T)[r][c]
-                gm[i][j] = fmaf(gr[i], mk[j], gm[i][j]);  // (G M)[r][c]
-            }
+        const float g = Gr[i * FP + k];
+        gw = fmaf(g, W0s[k * FP + c], gw);             // (G W0)[r][c]
+        gm = fmaf(g, Ms[k * FP + c], gm);              // (G M)[r][c]
+        xrc = fmaf(W0s[r * FP + k], Ms[c * FP + k], xrc);  // (W0 M^T)[r][c]
+        xcr = fmaf(W0s[c * FP + k], Ms[r * FP + k], xcr);  // (W0 M^T)[c][r]
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Xs[(r0 + i) * FP + c0 + j] = x[i][j];
-    __syncthreads();
-    __nv_bfloat16* ops = p.ops + (size_t)u * 8 * DD;
     const float en = p.eta_over_n;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = r0 + i, c = c0 + j;
-            const float ws = W0s[r * FP + c] - en * (gw[i][j] - Cts[c * FP + r]);  // C[r][c] = C^T[c][r]
-            const float a = Xs[r * FP + c] + Xs[c * FP + r];
-            const float m = Ms[r * FP + c];
-            p.dw0u[(size_t)u * DD + r * D + c] = m - en * gm[i][j];
-            put_hilo(ops, 0, r, c, ws);        // dQ[t][c'] = sum_b dO[t][b] W*[c'][b]
-            put_hilo(ops, 2, c, r, en * m);    // dV[t][c'] = sum_a K[t][a] (eta/N) M[a][c']
-            put_hilo(ops, 4, r, c, -en * a);   // dK[t][c'] += sum_a K[t][a] (-eta/N) A[a][c']  (A symmetric)
-            put_hilo(ops, 6, r, c, en * m);    // dK[t][c'] += sum_b V[t][b] (eta/N) M[c'][b]
-        }
+    const float ws = W0s[r * FP + c] - en * (gw - Cr[i * FP + c]);
+    const float a = xrc + xcr;
+    const float m = Ms[r * FP + c];
+    p.dw0u[(size_t)u * DD + r * D + c] = m - en * gm;
+    __nv_bfloat16* ops = p.ops + (size_t)u * 8 * DD;
+    put_hilo(ops, 0, r, c, ws);        // dQ[t][c'] = sum_b dO[t][b] W*[c'][b]
+    put_hilo(ops, 2, c, r, en * m);    // dV[t][c'] = sum_a K[t][a] (eta/N) M[a][c']
+    put_hilo(ops, 4, r, c, -en * a);   // dK[t][c'] += sum_a K[t][a] (-eta/N) A[a][c']  (A symmetric)
+    put_hilo(ops, 6, r, c, en * m);    // dK[t][c'] += sum_b V[t][b] (eta/N) M[c'][b]
 }
 
 // ----------------------------------------------------------------------------- apply -----

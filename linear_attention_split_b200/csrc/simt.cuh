@@ -442,7 +442,8 @@ __global__ void __launch_bounds__(TPB) linear_bwd_dw0(const float* __restrict__ 
     const int dd = d * d;
     if (e >= dd) return;
     float s = 0.f;
-    for (int b = 0; b < B; ++b) s += dw0u[((long long)b * H + h) * dd + e];
+#pragma unroll 8
+    for (int b = 0; b < B; ++b) s += dw0u[((long long)b * H + h) * dd + e];  // batch order
     dw0[(long long)h * dd + e] = s;
 }
 

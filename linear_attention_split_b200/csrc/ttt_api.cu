@@ -336,7 +336,7 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     fp.H = H;
     fp.S = pl.S;
     fp.eta_over_n = (float)((double)eta / (double)N);
-    lbw::finish_kernel<<<(unsigned)U, 256, lbw::f_smem_bytes(), st>>>(fp);
+    lbw::finish_kernel<<<dim3((unsigned)U, lbw::FBLOCKS), 256, lbw::f_smem_bytes(), st>>>(fp);
     lbw::AParams ap;
     ap.TT = pl.TT;
     ap.n_tiles = pl.n_tiles;
@@ -372,8 +372,8 @@ int linear_bwd_simt(const void* q, const void* k, const void* v, const float* w0
     return launched(4);
 }
 
-bool block_tc_ok(int C, int H, int dtype) {
-    return dtype == TTT_BF16 && C == blk::C && (C / H == 32 || C / H == 64) && C % H == 0;
+bool block_tc_ok(int C, int H, int Wg, int dtype) {
+    return dtype == TTT_BF16 && C == blk::C && (C / H == 32 || C / H == 64) && C % H == 0 && Wg <= blk::MAX_WG;
 }
 
 int check_common(const void* q, const void* k, const void* v, const void* out, int dtype, float eta) {
@@ -784,7 +784,7 @@ size_t ttt_vit3_block_workspace_bytes(int B, int Hg, int Wg, int C, int H, int d
     const size_t es = dtype == TTT_BF16 ? 2 : 4;
     const size_t t = align256((size_t)B * N * C * es);
     const size_t core = ttt_linear_fullbatch_workspace_bytes(B, H, (int)N, C / H, dtype);
-    const size_t z = block_tc_ok(C, H, dtype) ? 0 : align256((size_t)B * N * 2 * C * 4);
+    const size_t z = block_tc_ok(C, H, Wg, dtype) ? 0 : align256((size_t)B * N * 2 * C * 4);
     return 5 * t + core + z;
 }
 
@@ -810,14 +810,15 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
     void *q = w, *k = w + t, *v = w + 2 * t, *g = w + 3 * t, *o = w + 4 * t;
     void* core = w + 5 * t;
     const size_t core_bytes = ttt_linear_fullbatch_workspace_bytes(B, H, (int)N, d, dtype);
-    if (block_tc_ok(C, H, dtype)) {
+    if (block_tc_ok(C, H, Wg, dtype)) {
         DeviceInfo* dev = nullptr;
         if (int rc = current_device(&dev)) return rc;
         if (blk::p_smem_bytes() > dev->smem_optin || blk::o_smem_bytes() > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
         if ((rows + blk::MT - 1) / blk::MT > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
         const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-        CUtensorMap tx, tw, two;
+        CUtensorMap tx, tw, two, txw;
         if (!tmap_bf16_3d(&tx, x, blk::C, (int)rows, 1, blk::MT, sw) ||
+            !tmap_bf16_3d(&txw, x, blk::C, (int)rows, 1, blk::XW, sw) ||
             !tmap_bf16_box(&tw, wqkvg, 4 * blk::C, blk::C, 1, 64, 64, sw) ||
             !tmap_bf16_box(&two, wo, blk::C, 2 * blk::C, 1, 64, 2 * blk::C, sw))
             return TTT_ERR_CUDA;
@@ -852,7 +853,7 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         op.Wg = Wg;
         op.H = H;
         op.d = d;
-        blk::out_kernel<<<tiles, blk::THREADS, blk::o_smem_bytes(), st>>>(two, op);
+        blk::out_kernel<<<tiles, blk::O_THREADS, blk::o_smem_bytes(), st>>>(two, txw, op);
         return launched(1);
     }
     float* z = reinterpret_cast<float*>(static_cast<char*>(core) + core_bytes);
