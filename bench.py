@@ -597,7 +597,8 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=
                                                       2, None, 1.0, ws, stream), R, 5)
         res["minibatch_56x56_b64_e2"] = {"ms": ms, "tokens_per_s": 32 * 3136 / (ms / 1e3),
                                          "hbm_gbs_min_traffic": nb / (ms / 1e3) / 1e9, "kernels_per_call": 2,
-                                         "note": "CUDA-core kernels (one block per unit scans the chunks)"}
+                                         "note": "the scan's tensor-core recurrence in training mode (98 dependent "
+                                                 "steps), then the apply O = Q W_final"}
         del S, ws
     if only in (None, "block"):  # the ViT^3 block at the stage-1 width: B=32, 56x56, C=64, 2 heads of 32
         nb = 32 * 3136 * 64 * 2 * 2  # x in, y out

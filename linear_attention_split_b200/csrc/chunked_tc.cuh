@@ -29,6 +29,9 @@
 // A unidirectional scan (raster or reverse raster alone: the original, one-way TTT scan that
 // the Vision-TTT gist's bidirectional scan extends) runs one recurrence warp and one output
 // warp; the output warp rounds each chunk's O = Q_c W once and stores it, with nothing parked.
+// Training mode (mini-batch / multi-epoch inner training, the design-study options of the
+// ViT^3 blog) runs the raster recurrence over `steps` = epochs x nc chunks with no output warp
+// and no Q, and leaves W_final (fp32) in global memory for the apply pass.
 #pragma once
 #include "common.cuh"
 
@@ -56,6 +59,9 @@ struct Params {
     int H, N, nc;       // nc = N / 64
     int both;           // 1: both directions, summed; 0: direction `dir` alone
     int dir;            // the direction of a one-way scan: 0 raster, 1 reverse raster
+    int steps;          // recurrence steps: nc, or epochs x nc in training mode
+    float* wfin;        // training mode: W_final [U][64][64] fp32 (else nullptr)
+    float* wout;        // training mode: optional copy of W_final for the caller (or nullptr)
     float eta_over_b;
 };
 
@@ -80,7 +86,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int g = lane >> 2, t = lane & 3;  // fragment row / column-pair of this lane
     const int nc = p.nc;
     auto stage_ptr = [&](int dir, int s) { return ring + (dir * STAGES + s) * STAGE; };
-    auto chunk_of = [&](int dir, int step) { return dir == 0 ? step : nc - 1 - step; };
+    const bool train = p.wfin != nullptr;
+    const int steps = p.steps;
+    auto chunk_of = [&](int dir, int step) { return dir == 0 ? step % nc : nc - 1 - step; };
     auto wfr_ptr = [&](int dir, int b) { return reinterpret_cast<uint4*>(wfr + (dir * WBUF + b) * WFR); };
     auto active = [&](int dir) { return p.both || dir == p.dir; };
 
@@ -88,7 +96,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int d = 0; d < 2; ++d) {
             for (int s = 0; s < STAGES; ++s) {
                 mbar_init(&bars->full[d][s], 1);
-                mbar_init(&bars->empty[d][s], 2);  // the direction's recurrence and output warps
+                mbar_init(&bars->empty[d][s], train ? 1 : 2);  // the direction's recurrence (and output) warps
             }
             for (int b = 0; b < WBUF; ++b) {
                 mbar_init(&bars->wready[d][b], 1);
@@ -106,16 +114,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_v16);
-            for (int step = 0; step < nc; ++step)
+            for (int step = 0; step < steps; ++step)
                 for (int dir = 0; dir < 2; ++dir) {
                     if (!active(dir)) continue;
                     const int s = step % STAGES, use = step / STAGES;
                     if (use > 0) mbar_wait(&bars->empty[dir][s], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                     const int t0 = chunk_of(dir, step) * CB;
                     uint8_t* dst = stage_ptr(dir, s);
-                    mbar_expect_tx(&bars->full[dir][s], STAGE);
+                    mbar_expect_tx(&bars->full[dir][s], train ? STAGE - TILE : STAGE);
                     tma_load_3d(dst, &tm_k, 0, t0, u, &bars->full[dir][s]);
-                    tma_load_3d(dst + TILE, &tm_q, 0, t0, u, &bars->full[dir][s]);
+                    if (!train) tma_load_3d(dst + TILE, &tm_q, 0, t0, u, &bars->full[dir][s]);
                     tma_load_3d(dst + 2 * TILE, &tm_v16, col0, t0, u, &bars->full[dir][s]);
                 }
         }
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) load_a(smem_u32(stage_ptr(dir, 0)), i, ks, ka[i][ks]);
-        for (int step = 0; step < nc; ++step) {
+        for (int step = 0; step < steps; ++step) {
             const int s = step % STAGES;
             uint8_t* st = stage_ptr(dir, s);
             const uint32_t kb = smem_u32(st);
@@ -196,8 +204,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             // latency passes under the dW work
             const int b = step % WBUF, use = step / WBUF;
             const int sn = (step + 1) % STAGES;
-            const bool nf = step + 1 >= nc || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
-            const bool wf = use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
+            const bool nf = step + 1 >= steps || mbar_test_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1);
+            const bool wf = train || use == 0 || mbar_test_wait(&bars->wfree[dir][b], (use - 1) & 1);
             // K_i as B fragments of dW^T (k = tokens 16 i.., n = features): transposing loads;
             // (features 16 mt + 0..7) takes {kt[i][mt][0], [2]}, (16 mt + 8..15) {[1], [3]}
             uint32_t kt[4][4][4];
@@ -243,7 +251,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, V of this step consumed
             // the next step's K fragments load while this step's dW drains
-            if (step + 1 < nc) {
+            if (step + 1 < steps) {
                 if (!nf) mbar_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -255,6 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) wt[n][e] -= p.eta_over_b * dwt[n][e];
             make_a();
+            if (train) continue;  // training mode: no output per chunk
             // ---- hand W (after this step, fp32) to the output warp ---------------------------
             if (!wf) mbar_wait(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             {
@@ -264,6 +273,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->wready[dir][b]);
+        }
+        if (train) {  // W_final: wt[n] = {W[8n+2t][g], W[8n+2t+1][g], W[8n+2t][8+g], W[8n+2t+1][8+g]}
+            float* wf = p.wfin + (size_t)u * D * D + col0;
+            float* wo = p.wout ? p.wout + (size_t)u * D * D + col0 : nullptr;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int f = 8 * n + 2 * t;
+                const float v[4] = {wt[n][0], wt[n][1], wt[n][2], wt[n][3]};
+                const int fi[4] = {f, f + 1, f, f + 1}, ci[4] = {g, g, 8 + g, 8 + g};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    wf[fi[e] * D + ci[e]] = v[e];
+                    if (wo) wo[fi[e] * D + ci[e]] = v[e];
+                }
+            }
         }
         return;
     }
@@ -277,7 +301,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // parks before all additions.  The partner's parked partials (64 tokens x 16 columns,
     // fp32) are fetched PF steps ahead by one TMA box each into a ring of PF + 1 slots.
     const int dir = warp - 2;
-    if (!active(dir)) return;
+    if (train || !active(dir)) return;
     uint8_t* pk = pkr + dir * (PF + 1) * PKB;
     const int a0 = (nc & 1) && dir == 0 ? nc / 2 + 1 : nc / 2;  // first step that adds
     auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st

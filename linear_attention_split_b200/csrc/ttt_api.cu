@@ -616,7 +616,8 @@ size_t chunked_tc_ws(int B, int H, int N, int direction) {
 }
 
 int chunked_tc(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H, int N,
-               float eta, int direction, void* ws, cudaStream_t st) {
+               float eta, int direction, void* ws, cudaStream_t st, int epochs = 0, float* wfin = nullptr,
+               float* wout = nullptr) {
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     const int U = B * H;
@@ -629,6 +630,9 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
     p.nc = N / chk::CB;
     p.both = direction == 0 ? 1 : 0;
     p.dir = direction < 0 ? 1 : 0;
+    p.steps = wfin ? epochs * p.nc : p.nc;  // training mode: epochs over the chunks, no output
+    p.wfin = wfin;
+    p.wout = wout;
     p.eta_over_b = (float)((double)eta / (double)chk::CB);
     const int smem = 2 * chk::STAGES * chk::STAGE + 2 * chk::WBUF * chk::WFR + 2 * (chk::PF + 1) * chk::PKB +
                      (int)sizeof(chk::Bars) + 1024;
@@ -1036,6 +1040,13 @@ int ttt_linear_minibatch(const void* q, const void* k, const void* v, const floa
     if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
     float* wfin = static_cast<float*>(workspace);
     const float eta_over_b = (float)((double)eta / (double)chunk);
+    if (chunked_tc_ok(B, H, d, chunk, dtype)) {  // the tensor-core recurrence in training mode
+        if (int rc = chunked_tc(q, k, v, w0, out, B, H, N, eta, 1, nullptr, st, epochs, wfin, w_final)) return rc;
+        using T = __nv_bfloat16;
+        simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(static_cast<const T*>(q), wfin,
+                                                                                    static_cast<T*>(out), N, d);
+        return launched(1);
+    }
     if (dtype == TTT_BF16) {
         using T = __nv_bfloat16;
         if (cudaFuncSetAttribute(simt::minibatch_train<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
