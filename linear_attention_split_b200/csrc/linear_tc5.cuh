@@ -32,13 +32,12 @@
 //      counted on the owner's mbarrier); the owner adds the S contributions in rank order
 //      (deterministic, no atomics), forms W*^T rows = W0^T - (eta/N) grad^T in fp32 and sends
 //      them as bf16 hi + lo to every CTA of the cluster, again with st.async.
-//   4. Apply: Q tiles are loaded into the ring region, [O_hi | O_lo] = Q [W*_hi | W*_lo]
-//      (one N = 128 MMA chain per tile) into four TMEM buffers (all of TMEM: the Gram and
-//      W0^T G accumulators have been read by then); the Q tiles that fit are awaited while
-//      the exchange is in flight.  The epilogue warps form two groups of four (one warp per
-//      lane quarter) that take alternate tiles: add the two
-//      halves, write O as bf16 over the consumed Q tile, one TMA store per tile (rows >= N
-//      are clipped by the hardware).  A CTA ends once its last store has read shared memory;
+//   4. Apply: Q tiles are loaded into the ring region, O = Q W*_hi + Q W*_lo (two N = 64
+//      MMA chains accumulating into one 64-column buffer) in eight TMEM buffers (all of
+//      TMEM: the Gram and W0^T G accumulators have been read by then); the Q tiles that fit
+//      are awaited while the exchange is in flight.  The epilogue warps form two groups of
+//      four (one warp per lane quarter) that take alternate tiles: write O as bf16 over the
+//      consumed Q tile, one TMA store per tile (rows >= N are clipped by the hardware).  A CTA ends once its last store has read shared memory;
 //      the writes drain to memory while the next grid starts.
 // Every wait is bounded (common.cuh); after a wait has run out on the device, later waits give
 // up at once and the kernel runs to its normal end (results are then invalid and the host is
@@ -65,12 +64,13 @@ constexpr int FIXED_BYTES = 4 * OP_BYTES + RECV_BYTES;  // W0 hi/lo, W* hi/lo, r
 constexpr int TMEM_COLS = 512;
 constexpr int COL_A = 0;                       // Gram accumulator [C^T ; G]
 constexpr int COL_D = 64;                      // W0^T [G_hi | G_lo] (rows 0-63), 128 columns
-constexpr int COL_O = 0;                       // four [O_hi | O_lo] buffers of 128 columns (apply)
-constexpr int OBUFS = 4;
+constexpr int COL_O = 0;                       // eight O buffers of 64 columns (apply)
+constexpr int OBUFS = 8;
+static_assert((OBUFS & (OBUFS - 1)) == 0, "OBUFS is a power of two");
 constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
 constexpr uint32_t IDESC_WG = tc::idesc_bf16(128, 64, 0, 0);     // A K-major, B K-major
 constexpr uint32_t IDESC_WG2 = tc::idesc_bf16(128, 128, 0, 0);   // A K-major, B K-major, N = 128
-constexpr uint32_t IDESC_APPLY = tc::idesc_bf16(128, 128, 0, 0); // A K-major, B K-major
+constexpr uint32_t IDESC_APPLY = tc::idesc_bf16(128, 64, 0, 0);  // A K-major (Q), B K-major (W*^T)
 
 struct Params {
     const float* w0;    // [H][64][64]
@@ -276,24 +276,38 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::commit(&bars->dfull);
             }
 
-            // ---- apply: [O_hi | O_lo] = Q [W*_hi | W*_lo] per tile -----------------------------
+            // ---- apply: O = Q W*_hi + Q W*_lo per tile, accumulated in one 64-column buffer ---
             const int q_first = n_t < NQ ? n_t : NQ;  // tiles whose Q is loaded up front
             for (int t = 0; t < q_first; ++t) mbar_wait(&bars->qfull[t], 0, TTT_DEVERR_TIMEOUT_TMA);
             mbar_wait_cluster(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_PEER);   // the peers' W* rows
             mbar_wait(&bars->wlocal, 0, TTT_DEVERR_TIMEOUT_PEER);          // and this CTA's own
             fence_proxy_async_smem();  // W* rows were written by generic stores (local and st.async)
             tc::fence_after();
-            const uint64_t dws = tc::smem_desc(smem_u32(wsop), 16, 1024, 2);
-            for (int t = 0; t < n_t; ++t) {
-                const int b = t % OBUFS, qs = t % NQ;
-                if (t >= OBUFS) mbar_wait(&bars->tempty[b], (t / OBUFS - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-                if (t >= q_first) mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
-                tc::fence_after();
+            const uint64_t dwh = tc::smem_desc(smem_u32(wsop), 16, 1024, 2);
+            const uint64_t dwo = tc::smem_desc(smem_u32(wsop) + OP_BYTES, 16, 1024, 2);
+            auto apply_tile = [&](int t, int qs) {
+                const int b = t & (OBUFS - 1);
                 const uint64_t dq = tc::smem_desc(smem_u32(pool + qs * TILE_BYTES), 16, 1024, 2);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tmem + COL_O + b * 128, dq + 2 * ks, dws + 2 * ks, IDESC_APPLY, ks > 0 ? 1 : 0);
+                    tc::mma_bf16(tmem + COL_O + b * 64, dq + 2 * ks, dwh + 2 * ks, IDESC_APPLY, ks > 0 ? 1 : 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + COL_O + b * 64, dq + 2 * ks, dwo + 2 * ks, IDESC_APPLY, 1);
                 tc::commit(&bars->tfull[b]);
+            };
+            // Tiles whose Q tile has landed and whose TMEM buffer has never been used are issued
+            // by a loop with no waits in it (a bounded wait in the loop body, even one not taken,
+            // costs a few hundred cycles per tile between the MMA batches).
+            const int t_free = q_first < OBUFS ? q_first : OBUFS;
+            int t = 0;
+            for (; t < t_free; ++t) apply_tile(t, t);
+            for (; t < n_t; ++t) {
+                const int qs = t % NQ;
+                if (t >= OBUFS) mbar_wait(&bars->tempty[t & (OBUFS - 1)], (t / OBUFS - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                if (t >= q_first) mbar_wait(&bars->qfull[qs], (t / NQ) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                tc::fence_after();
+                apply_tile(t, qs);
             }
         }
         __syncwarp();
@@ -448,7 +462,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         cluster_arrive_release();  // every remote store of this thread has been issued
 
         // ---- O tiles: group h (one warp per lane quarter) takes tiles t = h, h + 2, ...:
-        //      TMEM -> (hi + lo) -> bf16 over the Q tile -> one TMA store per tile -------------
+        //      TMEM -> bf16 over the Q tile -> one TMA store per tile ------------------------------
         const bool storer = (q4 == 0 && lane == 0);
         for (int t = h; t < n_t; t += 2) {
             const int b = t % OBUFS, qs = t % NQ;
@@ -457,20 +471,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::fence_after();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                float oh[32], ol[32];
-                const uint32_t ob = lane_base + COL_O + b * 128 + half * 32;
-                tc::ld16(ob, &oh[0]);
-                tc::ld16(ob + 16, &oh[16]);
-                tc::ld16(ob + 64, &ol[0]);
-                tc::ld16(ob + 80, &ol[16]);
+                float o[32];
+                const uint32_t ob = lane_base + COL_O + b * 64 + half * 32;
+                tc::ld16(ob, &o[0]);
+                tc::ld16(ob + 16, &o[16]);
                 tc::wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     *reinterpret_cast<uint4*>(tile + swz<3>((uint32_t)row * ROWB + half * 64 + c * 16)) =
-                        make_uint4(pack_bf16(oh[8 * c] + ol[8 * c], oh[8 * c + 1] + ol[8 * c + 1]),
-                                   pack_bf16(oh[8 * c + 2] + ol[8 * c + 2], oh[8 * c + 3] + ol[8 * c + 3]),
-                                   pack_bf16(oh[8 * c + 4] + ol[8 * c + 4], oh[8 * c + 5] + ol[8 * c + 5]),
-                                   pack_bf16(oh[8 * c + 6] + ol[8 * c + 6], oh[8 * c + 7] + ol[8 * c + 7]));
+                        make_uint4(pack_bf16(o[8 * c], o[8 * c + 1]), pack_bf16(o[8 * c + 2], o[8 * c + 3]),
+                                   pack_bf16(o[8 * c + 4], o[8 * c + 5]), pack_bf16(o[8 * c + 6], o[8 * c + 7]));
             }
             tc::fence_before();
             __syncwarp();

@@ -107,3 +107,22 @@ def test_linear_zero_init_is_linear_attention():
     q, k, v = (inp[x].double() for x in ("q", "k", "v"))
     ref = (q @ (k.transpose(-1, -2) @ v)) / 3136
     assert_close(out, ref.numpy(), torch.bfloat16, "linear attention")
+
+
+# ---- few long units (the tensor-core kernel's cluster split at other token counts) -------
+@pytest.mark.parametrize("N", [3000, 1000, 6272, 3137])
+def test_linear_long_units_ragged(N):
+    """B=32 units of one head at ragged token counts: other tile heights and a partial last tile."""
+    check(32, 1, N, 64, "bf16", seed=N)
+
+
+@pytest.mark.parametrize("B,H", [(16, 2), (20, 2), (36, 1)])
+def test_linear_long_units_heads(B, H):
+    """Several heads per image (W0 differs between neighbouring units) and unit counts that
+    change the cluster size."""
+    check(B, H, 3136, 64, "bf16", seed=B * H)
+
+
+@pytest.mark.parametrize("eta", [0.0, -0.5])
+def test_linear_long_units_eta(eta):
+    check(32, 1, 3136, 64, "bf16", eta=eta, seed=3)
