@@ -11,10 +11,11 @@
 //   reduce : CTAs split each unit's tokens (as the forward does); per tile of V, K, Q, dO two
 //            tcgen05 MMAs accumulate [V | K]^T K (C^T and G) and [Q | dO]^T dO (M in its first
 //            64 rows) in TMEM; each CTA writes its partial G, C^T, M (fp32) to the workspace.
-//   finish : sixteen blocks per unit (four output rows each) add the partials in split order
-//            (deterministic) and form, in fp32 on the CUDA cores, W*, A and dW0_u; they write the
-//            four d x d right-hand operands of the token pass -- W*, (eta/N) M^T, -(eta/N) A,
-//            (eta/N) M -- each as bf16 hi + lo (row-major rows = output columns, i.e. K-major).
+//   finish : three blocks per unit, one per d x d product (G W0, W0 M^T, G M), add the partials
+//            in split order (deterministic) and form, in fp32 on the CUDA cores, W*, A and
+//            dW0_u; they write the four d x d right-hand operands of the token pass -- W*,
+//            (eta/N) M^T, -(eta/N) A, (eta/N) M -- each as bf16 hi + lo (row-major rows = output
+//            columns, i.e. K-major).
 //   apply  : per tile of dO, K, V: dQ = dO W*, dV = K (eta/N) M^T-operand, dK = K (-eta/N A) +
 //            V (eta/N M), each product taken as hi + lo into one 64-column TMEM accumulator;
 //            the outputs are written as bf16 over the consumed input tiles and stored by TMA.
@@ -155,74 +156,190 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 }
 
 // ----------------------------------------------------------------------------- finish ----
-// Grid (U, 16): block (u, rb) forms rows 4 rb .. 4 rb + 3 of W*, A and dW0_u (one output per
-// thread).  It adds the S partials (split order) of the four G rows and of all of M, takes W0
-// and the four C rows (columns of C^T), and writes its rows of the eight operands.
+// Grid (U, 3): block (u, j) forms one d x d product of unit u on the CUDA cores in fp32 --
+// j = 0: G W0,  j = 1: W0 M^T,  j = 2: G M -- with 256 threads, each holding a 4 x 4 tile of
+// it (outer products over k from two shared-memory operands laid out [k][row] and [k][col]:
+// two float4 reads per k), and writes what follows from that product:
+//   j = 0: W* = W0 - (eta/N)(G W0 - C)                          -> W* hi/lo
+//   j = 1: A = W0 M^T + (W0 M^T)^T                              -> -(eta/N) A hi/lo, and the
+//          M operands (eta/N) M^T hi/lo, (eta/N) M hi/lo
+//   j = 2: dW0_u = M - (eta/N) G M
+// The S partials are added in split order (deterministic), and every load of a matrix is
+// issued before the first of them is used (the partials were written by the previous kernel).
 struct FParams {
-    const float* part;     // [U][S][3][64][64]
+    const float* part;     // [U][S][3][64][64]: G, C^T, M
     const float* w0;       // [H][64][64]
     __nv_bfloat16* ops;    // [U][8][64][64]: W* hi/lo, (eta/N) M^T hi/lo, -(eta/N) A hi/lo, (eta/N) M hi/lo
     float* dw0u;           // [U][64][64]
-    int H, S;
+    int H, S;              // S <= 8
     float eta_over_n;
 };
-constexpr int FROWS = 4;                  // output rows per block
-constexpr int FBLOCKS = D / FROWS;        // blocks per unit
-constexpr int FP = D + 1;                 // padded row of the shared-memory matrices
-constexpr int f_smem_bytes() { return (2 * D * FP + 2 * FROWS * FP) * 4; }
+constexpr int FLD = D + 4;                // padded row of the shared-memory operands (float4 aligned)
+constexpr int f_smem_bytes() { return 2 * D * FLD * 4; }
 
-__device__ __forceinline__ void put_hilo(__nv_bfloat16* ops, int m, int row, int col, float x) {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    ops[(m * D + row) * D + col] = hi;
-    ops[((m + 1) * D + row) * D + col] = __float2bfloat16_rn(x - __bfloat162float(hi));
+// x[i] = sum over s < S (in order) of matrix `which` of the partials, float4 i of this thread
+// (elements 4 (tid + 256 i) ..): all S x 4 loads are issued before the first add
+__device__ __forceinline__ void f_load_sum(const float* part, int S, int which, int tid, float4 (&x)[4]) {
+    float4 v[8][4];
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+        if (s < S)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                v[s][i] = __ldg(reinterpret_cast<const float4*>(part + ((size_t)s * 3 + which) * DD) + tid + 256 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+        if (s < S)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[i].x += v[s][i].x;
+                x[i].y += v[s][i].y;
+                x[i].z += v[s][i].z;
+                x[i].w += v[s][i].w;
+            }
+}
+// float4 f of a d x d matrix (elements 4 f .. 4 f + 3 of row 4 f / 64) into an operand, as is
+// ([row][col]) or transposed
+__device__ __forceinline__ void f_put4(float* op, int f, float4 x, bool transposed) {
+    const int row = f >> 4, col = (f & 15) * 4;
+    if (transposed) {
+        op[col * FLD + row] = x.x;
+        op[(col + 1) * FLD + row] = x.y;
+        op[(col + 2) * FLD + row] = x.z;
+        op[(col + 3) * FLD + row] = x.w;
+    } else {
+        *reinterpret_cast<float4*>(op + row * FLD + col) = x;
+    }
+}
+__device__ __forceinline__ void put_hilo4(__nv_bfloat16* ops, int m, int row, int col, const float (&x)[4]) {
+    uint32_t hi[2], lo[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        const float2 hf = __bfloat1622float2(h);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+        hi[q] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[q] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    *reinterpret_cast<uint2*>(ops + ((size_t)m * D + row) * D + col) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(ops + ((size_t)(m + 1) * D + row) * D + col) = make_uint2(lo[0], lo[1]);
 }
 
 __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
     extern __shared__ float fsm[];
-    float* Ms = fsm;                  // all of M
-    float* W0s = Ms + D * FP;         // all of W0
-    float* Gr = W0s + D * FP;         // G rows r0 .. r0 + 3
-    float* Cr = Gr + FROWS * FP;      // C rows r0 .. r0 + 3 (C[r][c] = C^T[c][r])
-    const int u = blockIdx.x, r0 = blockIdx.y * FROWS, tid = threadIdx.x;
+    float* Aop = fsm;                 // [k][row]
+    float* Bop = fsm + D * FLD;       // [k][col]
+    const int u = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
     const float* W0 = p.w0 + (size_t)(u % p.H) * DD;
     const float* part = p.part + (size_t)u * p.S * 3 * DD;
-    for (int e = tid; e < DD; e += 256) {
-        float m = 0.f;
-        for (int s = 0; s < p.S; ++s) m += part[(size_t)s * 3 * DD + 2 * DD + e];  // split order
-        Ms[(e >> 6) * FP + (e & 63)] = m;
-        W0s[(e >> 6) * FP + (e & 63)] = W0[e];
-    }
+    // operands: j = 0: A[k][r] = G[k][r] (= G[r][k]: G = K^T K from exact bf16 products is
+    // symmetric), B = W0;  j = 1: A[k][r] = W0[r][k], B[k][c] = M[c][k];  j = 2: A = G, B = M
     {
-        const int i = tid >> 6, c = tid & 63;  // 4 rows x 64 columns
-        float g = 0.f, ct = 0.f;
-        for (int s = 0; s < p.S; ++s) {
-            g += part[(size_t)s * 3 * DD + (r0 + i) * D + c];
-            ct += part[(size_t)s * 3 * DD + DD + c * D + r0 + i];  // C^T[c][r]
+        float4 a[4], b[4];
+        if (j == 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = __ldg(reinterpret_cast<const float4*>(W0) + tid + 256 * i);
+        } else {
+            f_load_sum(part, p.S, 0, tid, a);
         }
-        Gr[i * FP + c] = g;
-        Cr[i * FP + c] = ct;
+        if (j == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) b[i] = __ldg(reinterpret_cast<const float4*>(W0) + tid + 256 * i);
+        } else {
+            f_load_sum(part, p.S, 2, tid, b);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f_put4(Aop, tid + 256 * i, a[i], j == 1);
+            f_put4(Bop, tid + 256 * i, b[i], j == 1);
+        }
     }
     __syncthreads();
-    const int i = tid >> 6, c = tid & 63, r = r0 + i;
-    float gw = 0.f, xrc = 0.f, xcr = 0.f, gm = 0.f;
-#pragma unroll 8
+    const int tr = tid >> 4, tc = tid & 15;  // rows 4 tr .. 4 tr + 3, columns 4 tc .. 4 tc + 3
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+#pragma unroll 4
     for (int k = 0; k < D; ++k) {
-        const float g = Gr[i * FP + k];
-        gw = fmaf(g, W0s[k * FP + c], gw);             // (G W0)[r][c]
-        gm = fmaf(g, Ms[k * FP + c], gm);              // (G M)[r][c]
-        xrc = fmaf(W0s[r * FP + k], Ms[c * FP + k], xrc);  // (W0 M^T)[r][c]
-        xcr = fmaf(W0s[c * FP + k], Ms[r * FP + k], xcr);  // (W0 M^T)[c][r]
+        const float4 av = *reinterpret_cast<const float4*>(Aop + k * FLD + 4 * tr);
+        const float4 bv = *reinterpret_cast<const float4*>(Bop + k * FLD + 4 * tc);
+        const float ax[4] = {av.x, av.y, av.z, av.w}, bx[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(ax[i], bx[q], acc[i][q]);
     }
     const float en = p.eta_over_n;
-    const float ws = W0s[r * FP + c] - en * (gw - Cr[i * FP + c]);
-    const float a = xrc + xcr;
-    const float m = Ms[r * FP + c];
-    p.dw0u[(size_t)u * DD + r * D + c] = m - en * gm;
     __nv_bfloat16* ops = p.ops + (size_t)u * 8 * DD;
-    put_hilo(ops, 0, r, c, ws);        // dQ[t][c'] = sum_b dO[t][b] W*[c'][b]
-    put_hilo(ops, 2, c, r, en * m);    // dV[t][c'] = sum_a K[t][a] (eta/N) M[a][c']
-    put_hilo(ops, 4, r, c, -en * a);   // dK[t][c'] += sum_a K[t][a] (-eta/N) A[a][c']  (A symmetric)
-    put_hilo(ops, 6, r, c, en * m);    // dK[t][c'] += sum_b V[t][b] (eta/N) M[c'][b]
+    const int c0 = 4 * tc;
+    if (j == 0) {
+        // C[r][c] = C^T[c][r]: for each column c, rows 4 tr .. 4 tr + 3 are one float4 of C^T
+        float4 cs[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cs[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < p.S; ++s) {
+            float4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[q] = __ldg(reinterpret_cast<const float4*>(part + ((size_t)s * 3 + 1) * DD + (c0 + q) * D + 4 * tr));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                cs[q].x += v[q].x;
+                cs[q].y += v[q].y;
+                cs[q].z += v[q].z;
+                cs[q].w += v[q].w;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * tr + i;
+            float w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float c = i == 0 ? cs[q].x : i == 1 ? cs[q].y : i == 2 ? cs[q].z : cs[q].w;
+                w[q] = Bop[r * FLD + c0 + q] - en * (acc[i][q] - c);
+            }
+            put_hilo4(ops, 0, r, c0, w);
+        }
+    } else if (j == 1) {
+        // A = P + P^T: the product goes through shared memory (over A's operand, now read)
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(Aop + (4 * tr + i) * FLD + c0) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * tr + i;
+            float a[4], mt[4], m[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = c0 + q;
+                a[q] = -en * (acc[i][q] + Aop[c * FLD + r]);
+                mt[q] = en * Bop[r * FLD + c];  // (eta/N) M[c][r]
+                m[q] = en * Bop[c * FLD + r];   // (eta/N) M[r][c]
+            }
+            put_hilo4(ops, 4, r, c0, a);
+            put_hilo4(ops, 2, r, c0, mt);
+            put_hilo4(ops, 6, r, c0, m);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * tr + i;
+            float4 o;
+            o.x = Bop[r * FLD + c0] - en * acc[i][0];
+            o.y = Bop[r * FLD + c0 + 1] - en * acc[i][1];
+            o.z = Bop[r * FLD + c0 + 2] - en * acc[i][2];
+            o.w = Bop[r * FLD + c0 + 3] - en * acc[i][3];
+            *reinterpret_cast<float4*>(p.dw0u + (size_t)u * DD + r * D + c0) = o;
+        }
+    }
 }
 
 // ----------------------------------------------------------------------------- apply -----

@@ -336,7 +336,7 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     fp.H = H;
     fp.S = pl.S;
     fp.eta_over_n = (float)((double)eta / (double)N);
-    lbw::finish_kernel<<<dim3((unsigned)U, lbw::FBLOCKS), 256, lbw::f_smem_bytes(), st>>>(fp);
+    lbw::finish_kernel<<<dim3((unsigned)U, 3), 256, lbw::f_smem_bytes(), st>>>(fp);
     lbw::AParams ap;
     ap.TT = pl.TT;
     ap.n_tiles = pl.n_tiles;
