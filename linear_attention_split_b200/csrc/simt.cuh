@@ -580,4 +580,80 @@ __global__ void __launch_bounds__(TPB) dwconv_prep2_bf16(const __nv_bfloat16* __
                    pack_bf16(acc[6], acc[7]));
 }
 
+// bf16, d = 64: block (column chunk, row strip) of unit blockIdx.y; thread (column, feature
+// group g) walks the strip's PS_ROWS rows with its 8 features' 72 filter taps in registers and
+// their 3 x 3 neighbourhood in a window that slides down one row per output token (three
+// 16-byte loads per output instead of nine).  A warp covers 4 consecutive tokens x 64 features:
+// 512 contiguous bytes per load and per store.  blockIdx.z picks K (0) or V (1).  The sums run
+// in the same order as dwconv_prep2_bf16 (tap row, tap column) with packed fp32 FMAs on feature
+// pairs (fma.rn.f32x2: an IEEE fma per lane), so both give the same values.
+constexpr int PS_ROWS = 8;
+__global__ void __launch_bounds__(256, 2) dwconv_prep_strip_bf16(const __nv_bfloat16* __restrict__ k,
+                                                              const __nv_bfloat16* __restrict__ v,
+                                                              const float* __restrict__ wk, const float* __restrict__ wv,
+                                                              __nv_bfloat16* __restrict__ kp,
+                                                              __nv_bfloat16* __restrict__ vp, int H, int Hg, int Wg) {
+    constexpr int D = 64;
+    const int g = threadIdx.x & 7, c = threadIdx.x >> 3;
+    const int nxc = (Wg + 31) / 32;
+    const int x = (int)(blockIdx.x % nxc) * 32 + c;
+    const int y0 = (int)(blockIdx.x / nxc) * PS_ROWS;
+    if (x >= Wg) return;  // no barrier below
+    const long long u = blockIdx.y;
+    const bool isv = blockIdx.z != 0;
+    const long long N = (long long)Hg * Wg;
+    const float* w = (isv ? wv : wk) + ((u % H) * D + g * 8) * 9;  // [8 features][9 taps]
+    uint64_t wr[4][9];  // taps of features (2i, 2i + 1) as packed fp32 pairs
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int t = 0; t < 9; ++t)
+            wr[i][t] = (uint64_t)__float_as_uint(__ldg(w + 2 * i * 9 + t)) |
+                       ((uint64_t)__float_as_uint(__ldg(w + (2 * i + 1) * 9 + t)) << 32);
+    const __nv_bfloat16* xu = (isv ? v : k) + u * N * D + g * 8;
+    __nv_bfloat16* ou = (isv ? vp : kp) + u * N * D + g * 8;
+    auto ld = [&](int yy, int xx) -> uint4 {
+        return (yy >= 0 && yy < Hg && xx >= 0 && xx < Wg)
+                   ? *reinterpret_cast<const uint4*>(xu + ((long long)yy * Wg + xx) * D)
+                   : make_uint4(0, 0, 0, 0);
+    };
+    uint4 win[3][3];  // rows y - 1, y, y + 1; columns x - 1, x, x + 1
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+        win[0][b] = ld(y0 - 1, x + b - 1);
+        win[1][b] = ld(y0, x + b - 1);
+        win[2][b] = ld(y0 + 1, x + b - 1);
+    }
+    const int y1 = min(y0 + PS_ROWS, Hg);
+    for (int y = y0; y < y1; ++y) {
+        uint4 nxt[3];  // row y + 2, requested before this row's arithmetic
+#pragma unroll
+        for (int b = 0; b < 3; ++b) nxt[b] = y + 1 < y1 ? ld(y + 2, x + b - 1) : make_uint4(0, 0, 0, 0);
+        uint64_t acc[4] = {0, 0, 0, 0};  // features (2i, 2i + 1), packed fp32
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {
+                const uint32_t wv4[4] = {win[a][b].x, win[a][b].y, win[a][b].z, win[a][b].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    // bf16 pair -> fp32 pair: low half to the high 16 bits of the first word
+                    const uint64_t f = (uint64_t)(wv4[i] << 16) | ((uint64_t)(wv4[i] & 0xffff0000u) << 32);
+                    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc[i]) : "l"(wr[i][a * 3 + b]), "l"(f));
+                }
+            }
+        *reinterpret_cast<uint4*>(ou + ((long long)y * Wg + x) * D) =
+            make_uint4(pack_bf16(__uint_as_float((uint32_t)acc[0]), __uint_as_float((uint32_t)(acc[0] >> 32))),
+                       pack_bf16(__uint_as_float((uint32_t)acc[1]), __uint_as_float((uint32_t)(acc[1] >> 32))),
+                       pack_bf16(__uint_as_float((uint32_t)acc[2]), __uint_as_float((uint32_t)(acc[2] >> 32))),
+                       pack_bf16(__uint_as_float((uint32_t)acc[3]), __uint_as_float((uint32_t)(acc[3] >> 32))));
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            win[0][b] = win[1][b];
+            win[1][b] = win[2][b];
+            win[2][b] = nxt[b];
+        }
+    }
+}
+
 }  // namespace simt

@@ -1101,7 +1101,15 @@ int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const f
     void* rest = w + 2 * align256((size_t)U * N * d * es);
     const size_t rest_bytes = workspace_bytes - 2 * align256((size_t)U * N * d * es);
     int prep_launches = 2;
-    if (dtype == TTT_BF16 && d % 8 == 0) {
+    if (dtype == TTT_BF16 && d == 64 && U <= 65535) {
+        using T = __nv_bfloat16;
+        const long long nblk = (long long)((Wg + 31) / 32) * ((Hg + simt::PS_ROWS - 1) / simt::PS_ROWS);
+        if (nblk > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+        simt::dwconv_prep_strip_bf16<<<dim3((unsigned)nblk, (unsigned)U, 2), 256, 0, st>>>(
+            static_cast<const T*>(k), static_cast<const T*>(v), wk, wv, static_cast<T*>(kp), static_cast<T*>(vp), H, Hg,
+            Wg);
+        prep_launches = 1;
+    } else if (dtype == TTT_BF16 && d % 8 == 0) {
         using T = __nv_bfloat16;
         dim3 grid = grid_units(U, N * (d / 8));
         grid.z = 2;
