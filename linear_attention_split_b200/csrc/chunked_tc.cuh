@@ -20,15 +20,19 @@
 // plain and transposing ldmatrix.  Nothing of the recurrence goes through shared memory, and
 // no other warp takes part in it.  The step's K, Q and the CTA's 16 V
 // columns arrive through a TMA ring filled by a producer warp (warp 4).  Each step the
-// recurrence warp hands its fp32 copy of W (4 KB) to an output warp of its direction (warps
-// 2, 3) through a small ring (wready / wfree); the output warp splits it into bf16 hi + lo B
-// fragments and computes O_c = Q_c W_hi + Q_c W_lo (W kept to 2^-17 in the output)
-// and the combine of the two directions, which meet in the middle: at step s < nc/2 each
-// direction parks its fp32 partial output for its chunk in the workspace; at step s >= nc/2
-// it adds the partner's parked partial, rounds once to bf16 and stores O (deterministic).
-// A unidirectional scan (raster or reverse raster alone: the original, one-way TTT scan that
-// the Vision-TTT gist's bidirectional scan extends) runs one recurrence warp and one output
-// warp; the output warp rounds each chunk's O = Q_c W once and stores it, with nothing parked.
+// recurrence warp hands its fp32 copy of W (4 KB) to the two output warps of its direction
+// (warps 2, 3 forward, 6, 7 backward; each takes two of the chunk's four 16-token tiles; a
+// warp runs on sub-partition warp % 4, so the recurrence warps 0 and 1 share theirs with
+// nothing but the mostly idle producer, and warp 5 has no work)
+// through a small ring (wready / wfree); an output warp splits W into bf16 hi + lo B
+// fragments and computes O = Q W_hi + Q W_lo for its 32 tokens (W kept to 2^-17 in the
+// output) and the combine of the two directions, which meet in the middle: at step s < nc/2
+// each direction parks its fp32 partial output for its chunk in the workspace; at step
+// s >= nc/2 it adds the partner's parked partial, rounds once to bf16 and stores O
+// (deterministic).  A unidirectional scan (raster or reverse raster alone: the original,
+// one-way TTT scan that the Vision-TTT gist's bidirectional scan extends) runs one recurrence
+// warp and its two output warps, which round each chunk's O = Q_c W once and store it, with
+// nothing parked.
 // Training mode (mini-batch / multi-epoch inner training, the design-study options of the
 // ViT^3 blog) runs the raster recurrence over `steps` = epochs x nc chunks with no output warp
 // and no Q, and leaves W_final (fp32) in global memory for the apply pass.
@@ -48,9 +52,11 @@ constexpr int STAGE = 2 * TILE + VT;    // one direction's data for one step
 constexpr int STAGES = 3;
 constexpr int WBUF = 4;                 // depth of the W hand-over ring
 constexpr int WFR = 32 * 32 * 4;        // one W slice (fp32 master copy): 32 registers x 32 lanes
-constexpr int THREADS = 5 * 32;         // 2 recurrence warps, 2 output warps, producer
+constexpr int THREADS = 8 * 32;         // 2 recurrence warps, 2 x 2 output warps, producer, one idle
+constexpr int OUT_TILES = 2;            // 16-token tiles of a chunk per output warp
 constexpr int PF = 2;                   // steps ahead that the partner's partials are copied
 constexpr int PKB = CB * NCOL * 4;       // one chunk's partials for the CTA's columns (4 KB)
+constexpr int PKH = PKB / 2;            // the half of them that one output warp adds
 
 struct Params {
     const float* w0;    // [H][64][64]
@@ -66,7 +72,7 @@ struct Params {
 };
 
 struct Bars {
-    uint64_t full[2][STAGES], empty[2][STAGES], wready[2][WBUF], wfree[2][WBUF], pfull[2][PF + 1];
+    uint64_t full[2][STAGES], empty[2][STAGES], wready[2][WBUF], wfree[2][WBUF], pfull[2][2][PF + 1];
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -96,18 +102,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int d = 0; d < 2; ++d) {
             for (int s = 0; s < STAGES; ++s) {
                 mbar_init(&bars->full[d][s], 1);
-                mbar_init(&bars->empty[d][s], train ? 1 : 2);  // the direction's recurrence (and output) warps
+                mbar_init(&bars->empty[d][s], train ? 1 : 3);  // the direction's recurrence (and output) warps
             }
             for (int b = 0; b < WBUF; ++b) {
                 mbar_init(&bars->wready[d][b], 1);
-                mbar_init(&bars->wfree[d][b], 1);
+                mbar_init(&bars->wfree[d][b], 2);  // both output warps of the direction
             }
-            for (int b = 0; b <= PF; ++b) mbar_init(&bars->pfull[d][b], 1);
+            for (int h = 0; h < 2; ++h)
+                for (int b = 0; b <= PF; ++b) mbar_init(&bars->pfull[d][h][b], 1);
         }
         mbar_fence_init();
     }
     __syncthreads();
 
+    if (warp == 5) return;  // keeps the output warps off the recurrence warps' sub-partitions
     if (warp == 4) {
         // ================================ producer ======================================
         if (lane == 0) {
@@ -300,15 +308,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     // the backward warp adds.  One barrier over the two output warps at step nc/2 orders all
     // parks before all additions.  The partner's parked partials (64 tokens x 16 columns,
     // fp32) are fetched PF steps ahead by one TMA box each into a ring of PF + 1 slots.
-    const int dir = warp - 2;
+    const int dir = warp >> 2, hf = warp & 1;  // warps 2, 3 / 6, 7; tiles 2 hf, 2 hf + 1 of each chunk
     if (train || !active(dir)) return;
-    uint8_t* pk = pkr + dir * (PF + 1) * PKB;
+    uint8_t* pk = pkr + dir * (PF + 1) * PKB + hf * PKH;
     const int a0 = (nc & 1) && dir == 0 ? nc / 2 + 1 : nc / 2;  // first step that adds
-    auto fetch = [&](int st) {  // parked partial of the chunk this direction visits at step st
+    auto fetch = [&](int st) {  // this warp's half of the parked partial of its step-st chunk
         if (lane == 0 && st < nc && st >= a0) {
             const int sl = (st - a0) % (PF + 1);
-            mbar_expect_tx(&bars->pfull[dir][sl], PKB);
-            tma_load_3d(pk + sl * PKB, &tm_park, col0, chunk_of(dir, st) * CB, u, &bars->pfull[dir][sl]);
+            mbar_expect_tx(&bars->pfull[dir][hf][sl], PKH);
+            tma_load_3d(pk + sl * PKB, &tm_park, col0, chunk_of(dir, st) * CB + hf * (CB / 2), u,
+                        &bars->pfull[dir][hf][sl]);
         }
     };
     for (int step = 0; step < nc; ++step) {
@@ -318,7 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t qb = smem_u32(stage_ptr(dir, s)) + TILE;
         uint32_t qa[4][4];
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) load_a(qb, 0, ks, qa[ks]);
+        for (int ks = 0; ks < 4; ++ks) load_a(qb, OUT_TILES * hf, ks, qa[ks]);
         mbar_wait(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
         // B fragments of W as bf16 hi + lo: k-step ks, column tile j (the recurrence warp's
         // W^T accumulator pairs, packed as its A fragments are)
@@ -349,13 +358,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->wfree[dir][b]);
-        float o[4][2][4];
+        float o[OUT_TILES][2][4];  // tile 2 hf + i
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < OUT_TILES; ++i) {
             uint32_t qn[4][4];
-            if (i < 3) {
+            if (i + 1 < OUT_TILES) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) load_a(qb, i + 1, ks, qn[ks]);
+                for (int ks = 0; ks < 4; ++ks) load_a(qb, OUT_TILES * hf + i + 1, ks, qn[ks]);
             }
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) mma_bf16(o[i][j], qa[ks], bw[hl][ks][j][0], bw[hl][ks][j][1]);
-            if (i < 3) {
+            if (i + 1 < OUT_TILES) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -377,12 +386,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // Q of this step consumed
         const size_t tok0 = (size_t)u * p.N + (size_t)chunk_of(dir, step) * CB;
-        auto out_index = [&](int i, int j, int h) {
-            return (tok0 + 16 * i + g + 8 * h) * D + col0 + 8 * j + 2 * t;
+        auto out_index = [&](int i, int j, int h) {  // i: this warp's tile 2 hf + i
+            return (tok0 + 16 * (OUT_TILES * hf + i) + g + 8 * h) * D + col0 + 8 * j + 2 * t;
         };
         if (!p.both) {  // one-way scan: this is the chunk's output
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < OUT_TILES; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -392,7 +401,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (step < a0) {  // first visit: park the fp32 partial
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < OUT_TILES; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -403,25 +412,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (step == nc / 2) {
             // every park is written, and visible to the tensor-copy reads that follow
             asm volatile("fence.proxy.async.global;" ::: "memory");
-            asm volatile("bar.sync 1, 64;" ::: "memory");
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // the four output warps
 #pragma unroll
             for (int k = 0; k < PF; ++k) fetch(a0 + k);
         }
         if (step >= a0) {
             // second visit: add the partner's partial, round once, store O.  Every read of the
             // slot is issued before the first store, so that no read waits behind a store.
-            mbar_wait(&bars->pfull[dir][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1, TTT_DEVERR_TIMEOUT_TMA);
+            mbar_wait(&bars->pfull[dir][hf][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1,
+                      TTT_DEVERR_TIMEOUT_TMA);
             const float* other = reinterpret_cast<const float*>(pk + ((step - a0) % (PF + 1)) * PKB);
-            float2 x[4][2][2];
+            float2 x[OUT_TILES][2][2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < OUT_TILES; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         x[i][j][h] = *reinterpret_cast<const float2*>(other + (16 * i + g + 8 * h) * NCOL + 8 * j + 2 * t);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < OUT_TILES; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll

@@ -652,11 +652,13 @@ int chunked_tc(const void* q, const void* k, const void* v, const float* w0, voi
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return TTT_ERR_CUDA;
-        // parked partials (fp32 [U][N][64]): box of 16 columns x 64 tokens, no swizzle (a one-way
-        // scan parks nothing and never uses this map; it is encoded over `out` then)
+        // parked partials (fp32 [U][N][64]): box of 16 columns x 32 tokens (one output warp's
+        // half of a chunk), no swizzle (a one-way scan parks nothing and never uses this map; it
+        // is encoded over `out` then)
         cuuint64_t pstrides[2] = {256, (cuuint64_t)N * 256};
+        cuuint32_t pbox[3] = {chk::NCOL, chk::CB / 2, 1};
         void* pbase = ws ? ws : out;
-        if (fn(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, pbase, dims, pstrides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        if (fn(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, pbase, dims, pstrides, pbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return TTT_ERR_CUDA;
