@@ -39,6 +39,7 @@ constexpr int R_STAGE = 4 * TILE;         // V, K, Q, dO
 constexpr int R_THREADS = 64 + 128;       // producer, issuer, 4 epilogue warps
 constexpr uint32_t IDESC_GRAM = tc::idesc_bf16(128, 64, 1, 1);  // A MN-major, B MN-major
 constexpr uint32_t IDESC_N64 = tc::idesc_bf16(128, 64, 0, 0);   // A K-major, B K-major
+constexpr uint32_t IDESC_N128 = tc::idesc_bf16(128, 128, 0, 0); // A K-major, B K-major
 
 struct RParams {
     float* part;      // [U][S][3][64][64]: G, C^T, M
@@ -169,12 +170,17 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 struct FParams {
     const float* part;     // [U][S][3][64][64]: G, C^T, M
     const float* w0;       // [H][64][64]
-    __nv_bfloat16* ops;    // [U][8][64][64]: W* hi/lo, (eta/N) M^T hi/lo, -(eta/N) A hi/lo, (eta/N) M hi/lo
+    __nv_bfloat16* ops;    // [U][8][64][64]: the slots OP_* below (W*, (eta/N) M^T, -(eta/N) A, (eta/N) M, hi and lo)
     float* dw0u;           // [U][64][64]
     int H, S;              // S <= 8
     float eta_over_n;
 };
 constexpr int FLD = D + 4;                // padded row of the shared-memory operands (float4 aligned)
+// Slots of the eight right-hand operands (64 x 64 bf16 each, [U][8][64][64]).  (eta/N) M^T and
+// -(eta/N) A sit side by side, hi next to hi and lo next to lo, so that K [M^T-op | A-op] is one
+// N = 128 product giving dV and the first term of dK in adjacent accumulator columns.
+constexpr int OP_WS_HI = 0, OP_WS_LO = 1, OP_MT_HI = 2, OP_A_HI = 3, OP_MT_LO = 4, OP_A_LO = 5, OP_M_HI = 6,
+              OP_M_LO = 7;
 constexpr int f_smem_bytes() { return 2 * D * FLD * 4; }
 
 // x[i] = sum over s < S (in order) of matrix `which` of the partials, float4 i of this thread
@@ -213,7 +219,7 @@ __device__ __forceinline__ void f_put4(float* op, int f, float4 x, bool transpos
         *reinterpret_cast<float4*>(op + row * FLD + col) = x;
     }
 }
-__device__ __forceinline__ void put_hilo4(__nv_bfloat16* ops, int m, int row, int col, const float (&x)[4]) {
+__device__ __forceinline__ void put_hilo4(__nv_bfloat16* ops, int mh, int ml, int row, int col, const float (&x)[4]) {
     uint32_t hi[2], lo[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -223,8 +229,8 @@ __device__ __forceinline__ void put_hilo4(__nv_bfloat16* ops, int m, int row, in
         hi[q] = *reinterpret_cast<const uint32_t*>(&h);
         lo[q] = *reinterpret_cast<const uint32_t*>(&l);
     }
-    *reinterpret_cast<uint2*>(ops + ((size_t)m * D + row) * D + col) = make_uint2(hi[0], hi[1]);
-    *reinterpret_cast<uint2*>(ops + ((size_t)(m + 1) * D + row) * D + col) = make_uint2(lo[0], lo[1]);
+    *reinterpret_cast<uint2*>(ops + ((size_t)mh * D + row) * D + col) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(ops + ((size_t)ml * D + row) * D + col) = make_uint2(lo[0], lo[1]);
 }
 
 __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
                 const float c = i == 0 ? cs[q].x : i == 1 ? cs[q].y : i == 2 ? cs[q].z : cs[q].w;
                 w[q] = Bop[r * FLD + c0 + q] - en * (acc[i][q] - c);
             }
-            put_hilo4(ops, 0, r, c0, w);
+            put_hilo4(ops, OP_WS_HI, OP_WS_LO, r, c0, w);
         }
     } else if (j == 1) {
         // A = P + P^T: the product goes through shared memory (over A's operand, now read)
@@ -324,9 +330,9 @@ __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
                 mt[q] = en * Bop[r * FLD + c];  // (eta/N) M[c][r]
                 m[q] = en * Bop[c * FLD + r];   // (eta/N) M[r][c]
             }
-            put_hilo4(ops, 4, r, c0, a);
-            put_hilo4(ops, 2, r, c0, mt);
-            put_hilo4(ops, 6, r, c0, m);
+            put_hilo4(ops, OP_A_HI, OP_A_LO, r, c0, a);
+            put_hilo4(ops, OP_MT_HI, OP_MT_LO, r, c0, mt);
+            put_hilo4(ops, OP_M_HI, OP_M_LO, r, c0, m);
         }
     } else {
 #pragma unroll
@@ -435,20 +441,21 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                 const uint64_t dk = tc::smem_desc(sb + TILE, 16, 1024, 2);
                 const uint64_t dv = tc::smem_desc(sb + 2 * TILE, 16, 1024, 2);
                 const uint32_t acc0 = tmem + b * 256;
-                // dQ (columns 0-63), dV (64-127), dK (128-191); each right operand as hi + lo
+                // dQ (columns 0-63), then [dV | dK] (64-191) = K [M^T-op | A-op] as one N = 128
+                // product, then dK += V M-op; each right operand as hi + lo
 #pragma unroll
                 for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const int acc = (hl > 0 || ks > 0) ? 1 : 0;
-                        tc::mma_bf16(acc0, dg + 2 * ks, od[0 + hl] + 2 * ks, IDESC_N64, acc);
-                        tc::mma_bf16(acc0 + 64, dk + 2 * ks, od[2 + hl] + 2 * ks, IDESC_N64, acc);
-                        tc::mma_bf16(acc0 + 128, dk + 2 * ks, od[4 + hl] + 2 * ks, IDESC_N64, acc);
+                        tc::mma_bf16(acc0, dg + 2 * ks, od[hl ? OP_WS_LO : OP_WS_HI] + 2 * ks, IDESC_N64, acc);
+                        tc::mma_bf16(acc0 + 64, dk + 2 * ks, od[hl ? OP_MT_LO : OP_MT_HI] + 2 * ks, IDESC_N128, acc);
                     }
 #pragma unroll
                 for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) tc::mma_bf16(acc0 + 128, dv + 2 * ks, od[6 + hl] + 2 * ks, IDESC_N64, 1);
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc::mma_bf16(acc0 + 128, dv + 2 * ks, od[hl ? OP_M_LO : OP_M_HI] + 2 * ks, IDESC_N64, 1);
                 tc::commit(&bars->tfull[b]);
             }
         }
