@@ -131,7 +131,8 @@ struct OBars {
 };
 constexpr int o_smem_bytes() { return 2 * ZT + XW * ROWB + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
 
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
+// 1 / (1 + e^-z) with the fast exponential and the fast (approximate, ~2 ulp) division
+__device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 // eight fp32 values -> bf16 hi and lo = bf16(x - hi), packed
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
     uint32_t h[4], l[4];
@@ -163,7 +164,11 @@ __global__ void __launch_bounds__(O_THREADS, 1)
         mbar_init(&bars->done, 1);
         mbar_fence_init();
     }
-    for (int e = threadIdx.x; e < C * 9; e += O_THREADS) wcs[e] = p.wc[e];
+    // taps regrouped as [8-channel chunk][tap][8 channels]: one tap of a chunk is two float4
+    for (int e = threadIdx.x; e < C * 9; e += O_THREADS) {
+        const int ch = e / 9, tap = e % 9;
+        wcs[((ch >> 3) * 9 + tap) * 8 + (ch & 7)] = p.wc[e];
+    }
     if (warp == O_WARPS) tc::alloc(&bars->tmem_base, 64);
     tc::fence_before();
     __syncthreads();
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(O_THREADS, 1)
                     m[2 * i + 1] = of.y * sigmoidf_(gf.y);
                 }
                 split8(m, mz, mzl);
-                float acc[8] = {};
+                uint64_t acc2[4] = {0, 0, 0, 0};  // channel pairs (2i, 2i + 1), packed fp32
 #pragma unroll
                 for (int a = 0; a < 3; ++a)
 #pragma unroll
@@ -232,14 +237,26 @@ __global__ void __launch_bounds__(O_THREADS, 1)
                         if (yy < 0 || yy >= p.Hg || xx < 0 || xx >= p.Wg) continue;
                         const int wr = wrow + (a - 1) * p.Wg + (bb - 1);  // same image: inside the window
                         const uint4 raw = *reinterpret_cast<const uint4*>(xw + wr * ROWB + ((chunk ^ (wr & 7)) << 4));
-                        const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                        const float4* wt = reinterpret_cast<const float4*>(wcs + (chunk * 9 + a * 3 + bb) * 8);
+                        const float4 w0 = wt[0], w1 = wt[1];
+                        const uint64_t wp[4] = {
+                            (uint64_t)__float_as_uint(w0.x) | ((uint64_t)__float_as_uint(w0.y) << 32),
+                            (uint64_t)__float_as_uint(w0.z) | ((uint64_t)__float_as_uint(w0.w) << 32),
+                            (uint64_t)__float_as_uint(w1.x) | ((uint64_t)__float_as_uint(w1.y) << 32),
+                            (uint64_t)__float_as_uint(w1.z) | ((uint64_t)__float_as_uint(w1.w) << 32)};
+                        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 f = __bfloat1622float2(r2[i]);
-                            acc[2 * i] = fmaf(wcs[(c + 2 * i) * 9 + a * 3 + bb], f.x, acc[2 * i]);
-                            acc[2 * i + 1] = fmaf(wcs[(c + 2 * i + 1) * 9 + a * 3 + bb], f.y, acc[2 * i + 1]);
+                        for (int i = 0; i < 4; ++i) {  // bf16 pair -> fp32 pair, then one fma per lane
+                            const uint64_t f = (uint64_t)(rw[i] << 16) | ((uint64_t)(rw[i] & 0xffff0000u) << 32);
+                            asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2[i]) : "l"(wp[i]), "l"(f));
                         }
                     }
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] = __uint_as_float((uint32_t)acc2[i]);
+                    acc[2 * i + 1] = __uint_as_float((uint32_t)(acc2[i] >> 32));
+                }
                 split8(acc, dz, dzl);
             }
             const uint32_t off = swz<3>((uint32_t)row * ROWB + c * 2);
