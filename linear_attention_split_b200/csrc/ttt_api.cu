@@ -12,6 +12,8 @@
 #include <mutex>
 #include <algorithm>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ttt.h"
 #include "common.cuh"
 #include "simt.cuh"
@@ -37,6 +39,15 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_lock;
+
+// A host-side NVTX range around one entry point's launches (profilers show each call as a
+// named range; without a tool attached it costs a branch).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int current_device(DeviceInfo** info) {
     int dev = 0;
@@ -767,6 +778,7 @@ size_t ttt_linear_fullbatch_workspace_bytes(int B, int H, int N, int d, int dtyp
 int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star,
                          int B, int H, int N, int d, float eta, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_fullbatch");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w0 || !aligned16(w0) || (w_star && !aligned16(w_star))) return TTT_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return TTT_ERR_INVALID_ARG;
@@ -797,6 +809,7 @@ size_t ttt_vit3_block_workspace_bytes(int B, int Hg, int Wg, int C, int H, int d
 int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const float* wc, const void* wo, void* y,
                    int B, int Hg, int Wg, int C, int H, float eta, int dtype, void* workspace,
                    size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_vit3_block");
     if (!x || !wqkvg || !w0 || !wc || !wo || !y) return TTT_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(wqkvg) || !aligned16(w0) || !aligned16(wc) || !aligned16(wo) || !aligned16(y))
         return TTT_ERR_INVALID_ARG;
@@ -912,6 +925,7 @@ size_t ttt_linear_fullbatch_bwd_workspace_bytes(int B, int H, int N, int d, int 
 int ttt_linear_fullbatch_bwd(const void* q, const void* k, const void* v, const float* w0, const void* dout,
                              void* dq, void* dk, void* dv, float* dw0, int B, int H, int N, int d, float eta,
                              int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_fullbatch_bwd");
     if (int rc = check_common(q, k, v, dout, dtype, eta)) return rc;
     if (!dq || !dk || !dv || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return TTT_ERR_INVALID_ARG;
     if (!w0 || !dw0 || !aligned16(w0) || !aligned16(dw0)) return TTT_ERR_INVALID_ARG;
@@ -937,6 +951,7 @@ size_t ttt_dwconv_fullbatch_workspace_bytes(int B, int Hg, int Wg, int C, int dt
 int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star,
                          int B, int Hg, int Wg, int C, float eta, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_dwconv_fullbatch");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w0 || !aligned16(w0) || (w_star && !aligned16(w_star))) return TTT_ERR_INVALID_ARG;
     if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return TTT_ERR_INVALID_ARG;
@@ -959,6 +974,7 @@ size_t ttt_mlp_fullbatch_workspace_bytes(int B, int H, int N, int d, int hidden,
 int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* w1, const float* w2, void* out,
                       float* w1_star, float* w2_star, int B, int H, int N, int d, int hidden, float eta, int dtype,
                       void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_mlp_fullbatch");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w1 || !w2 || !aligned16(w1) || !aligned16(w2)) return TTT_ERR_INVALID_ARG;
     if ((w1_star && !aligned16(w1_star)) || (w2_star && !aligned16(w2_star))) return TTT_ERR_INVALID_ARG;
@@ -985,6 +1001,7 @@ size_t ttt_linear_chunked_workspace_bytes(int B, int H, int N, int d, int chunk,
 int ttt_linear_chunked(const void* q, const void* k, const void* v, const float* w0, void* out, int B, int H,
                        int N, int d, int chunk, float eta, int direction, int dtype, void* workspace,
                        size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_chunked");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w0 || !aligned16(w0)) return TTT_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0) return TTT_ERR_INVALID_ARG;
@@ -1007,6 +1024,7 @@ size_t ttt_linear_chunked_bidir_workspace_bytes(int B, int H, int N, int d, int 
 int ttt_linear_chunked_bidir(const void* q, const void* k, const void* v, const float* w0, void* out, int B,
                              int H, int N, int d, int chunk, float eta, int dtype, void* workspace,
                              size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_chunked_bidir");
     return ttt_linear_chunked(q, k, v, w0, out, B, H, N, d, chunk, eta, 0, dtype, workspace, workspace_bytes,
                               stream);
 }
@@ -1022,6 +1040,7 @@ size_t ttt_linear_minibatch_workspace_bytes(int B, int H, int N, int d, int chun
 int ttt_linear_minibatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_final,
                          int B, int H, int N, int d, int chunk, int epochs, float eta, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_minibatch");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w0 || !aligned16(w0) || (w_final && !aligned16(w_final))) return TTT_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || chunk <= 0 || N % chunk != 0 || epochs <= 0)
@@ -1085,6 +1104,7 @@ size_t ttt_linear_chunked_conv_workspace_bytes(int B, int H, int Hg, int Wg, int
 int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const float* w0, const float* wk,
                             const float* wv, void* out, int B, int H, int Hg, int Wg, int d, int chunk, float eta,
                             int direction, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("ttt_linear_chunked_conv");
     if (int rc = check_common(q, k, v, out, dtype, eta)) return rc;
     if (!w0 || !wk || !wv || !aligned16(w0) || !aligned16(wk) || !aligned16(wv)) return TTT_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || d <= 0 || chunk <= 0) return TTT_ERR_INVALID_ARG;
