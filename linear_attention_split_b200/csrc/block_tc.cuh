@@ -9,8 +9,10 @@
 //     y = [O * sigmoid(G) | dwconv3x3(x)] Wo
 // Two kernels around the core (the full-batch step needs every token's K and V before any
 // output, so the core is a kernel of its own):
-//   proj : per 128-token tile, x (TMA) times Wqkvg (resident, MN-major) into 256 TMEM columns;
-//          the epilogue writes Q, K, V head-split [B, H, N, d] and G [B, N, C] in bf16.
+//   proj : persistent, one CTA per SM looping over the 128-token tiles: x tiles through a TMA
+//          ring, Wqkvg resident (MN-major), x Wqkvg into one of two 256-column TMEM
+//          accumulators, so that the epilogue -- Q, K, V head-split [B, H, N, d] and G [B, N, C]
+//          in bf16 -- of one tile overlaps the loads and the MMAs of the next.
 //   out  : per 128-token tile, four warps build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128,
 //          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows
 //          (16-byte loads, all issued up front), the conv from a window of x rows that one TMA
@@ -33,7 +35,8 @@ constexpr int WO = 2 * C * C * 2;       // Wo, 16 KB
 constexpr int XW = 256;                 // rows of the x window (tile + halo)
 constexpr int MAX_WG = (XW - MT) / 2 - 1;  // widest grid the window covers (63)
 constexpr int P_WARPS = 8;              // proj: eight epilogue warps (row quarter x column half)
-constexpr int THREADS = 32 * P_WARPS + 32;  // + one issuer warp
+constexpr int THREADS = 32 * P_WARPS + 64;  // + one MMA issuer warp and one x-tile producer warp
+constexpr int PXS = 4;                  // proj: x tile ring slots
 constexpr int O_WARPS = 16;             // out: sixteen Z / epilogue warps (row quarter x 16 channels)
 constexpr int O_THREADS = 32 * O_WARPS + 32;
 
@@ -43,77 +46,120 @@ struct PParams {
     int N, H, d;
 };
 struct PBars {
-    uint64_t full, done;
+    uint64_t wfull, xfull[PXS], xempty[PXS], done[2], tfree[2];
     uint32_t tmem_base;
 };
-constexpr int p_smem_bytes() { return XT + WQ + (int)sizeof(PBars) + 1024; }
+constexpr int p_smem_bytes() { return PXS * XT + WQ + (int)sizeof(PBars) + 1024; }
 
 __global__ void __launch_bounds__(THREADS, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const PParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ws = xs + XT;
+    uint8_t* ws = xs + PXS * XT;
     PBars* bars = reinterpret_cast<PBars*>(ws + WQ);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row0 = (long long)blockIdx.x * MT;
+    const long long ntiles = (p.rows + MT - 1) / MT;
+    const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA (>= 1)
+    auto row0_of = [&](int j) { return ((long long)blockIdx.x + (long long)j * gridDim.x) * MT; };
     if (threadIdx.x == 32 * P_WARPS) {
-        mbar_init(&bars->full, 1);
-        mbar_init(&bars->done, 1);
+        mbar_init(&bars->wfull, 1);
+        for (int s = 0; s < PXS; ++s) {
+            mbar_init(&bars->xfull[s], 1);
+            mbar_init(&bars->xempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->done[b], 1);
+            mbar_init(&bars->tfree[b], P_WARPS);
+        }
         mbar_fence_init();
     }
-    if (warp == P_WARPS) tc::alloc(&bars->tmem_base, 256);
+    if (warp == P_WARPS) tc::alloc(&bars->tmem_base, 512);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars->tmem_base;
-    if (warp == P_WARPS) {
+    if (warp == P_WARPS + 1) {
+        // ================================ producer: weights, then the x tiles ================
         if (lane == 0) {
-            mbar_expect_tx(&bars->full, XT + WQ);  // out-of-range rows are zero-filled and counted
-            tma_load_3d(xs, &tm_x, 0, (int)row0, 0, &bars->full);
+            mbar_expect_tx(&bars->wfull, WQ);
 #pragma unroll
-            for (int a = 0; a < 4; ++a) tma_load_3d(ws + a * 8192, &tm_w, a * 64, 0, 0, &bars->full);
-            mbar_wait(&bars->full, 0, TTT_DEVERR_TIMEOUT_TMA);
-            tc::fence_after();
-            const uint32_t xa = smem_u32(xs), wa = smem_u32(ws);
+            for (int a = 0; a < 4; ++a) tma_load_3d(ws + a * 8192, &tm_w, a * 64, 0, 0, &bars->wfull);
+            for (int j = 0; j < nj; ++j) {
+                const int s = j % PXS, use = j / PXS;
+                if (use > 0) mbar_wait(&bars->xempty[s], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                mbar_expect_tx(&bars->xfull[s], XT);  // out-of-range rows are zero-filled and counted
+                tma_load_3d(xs + s * XT, &tm_x, 0, (int)row0_of(j), 0, &bars->xfull[s]);
+            }
+        }
+    } else if (warp == P_WARPS) {
+        // ================================ MMA issuer ===========================================
+        if (lane == 0) {
+            mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
+            const uint32_t wa = smem_u32(ws);
             constexpr uint32_t ID = tc::idesc_bf16(128, 256, 0, 1);  // A K-major, B MN-major, N = 256
+            for (int j = 0; j < nj; ++j) {
+                const int s = j % PXS, b = j & 1;
+                mbar_wait(&bars->xfull[s], (j / PXS) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                if (j >= 2) mbar_wait(&bars->tfree[b], ((j >> 1) - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
+                const uint32_t xa = smem_u32(xs + s * XT);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16(tmem, tc::smem_desc(xa + ks * 32, 16, 1024, 2), tc::smem_desc(wa + ks * 2048, 8192, 1024, 2),
-                             ID, ks > 0 ? 1 : 0);
-            tc::commit(&bars->done);
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tmem + b * 256, tc::smem_desc(xa + ks * 32, 16, 1024, 2),
+                                 tc::smem_desc(wa + ks * 2048, 8192, 1024, 2), ID, ks > 0 ? 1 : 0);
+                tc::commit(&bars->done[b]);
+                tc::commit(&bars->xempty[s]);  // the slot may take a later tile
+            }
         }
     } else {
+        // ================================ epilogue (eight warps) ===============================
         const int q4 = warp & 3, ch = warp >> 2;  // lane quarter, column half (Q, K | V, G)
         const int row = q4 * 32 + lane;
-        const long long R = row0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-        mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
-        tc::fence_after();
-        const long long b = R / p.N, t = R % p.N;
+        for (int j = 0; j < nj; ++j) {
+            const int b = j & 1;
+            const long long R = row0_of(j) + row;
+            const long long bi = R / p.N, t = R % p.N;
+            mbar_wait(&bars->done[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+            tc::fence_after();
+            // this warp's 128 columns in two TMEM round trips of four 16-column chunks
 #pragma unroll 1
-        for (int j0 = ch * 2 * C; j0 < (ch + 1) * 2 * C; j0 += 16) {
-            float v[16];
-            tc::ld16(lane_base + j0, v);
-            tc::wait_ld();
-            if (R >= p.rows) continue;
-            const int which = j0 / C, c = j0 % C;
-            __nv_bfloat16* dst;
-            if (which == 3) {
-                dst = p.g + R * C + c;
-            } else {
-                const int h = c / p.d, e = c % p.d;
-                __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : p.v;
-                dst = base + ((b * p.H + h) * p.N + t) * p.d + e;
+            for (int g4 = 0; g4 < 2; ++g4) {
+                float v[4][16];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) tc::ld16(lane_base + b * 256 + ch * 2 * C + (4 * g4 + c4) * 16, v[c4]);
+                tc::wait_ld();
+                if (g4 == 1) {  // the accumulator has been read: the next tile but one may use it
+                    tc::fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->tfree[b]);
+                }
+                if (R >= p.rows) continue;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int j0 = ch * 2 * C + (4 * g4 + c4) * 16;
+                    const int which = j0 / C, c = j0 % C;
+                    __nv_bfloat16* dst;
+                    if (which == 3) {
+                        dst = p.g + R * C + c;
+                    } else {
+                        const int h = c / p.d, e = c % p.d;
+                        __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : p.v;
+                        dst = base + ((bi * p.H + h) * p.N + t) * p.d + e;
+                    }
+                    const float* x = v[c4];
+                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+                    d4[0] = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                       pack_bf16(x[6], x[7]));
+                    d4[1] = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]),
+                                       pack_bf16(x[14], x[15]));
+                }
             }
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-            d4[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-            d4[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
-                               pack_bf16(v[14], v[15]));
         }
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == P_WARPS) tc::dealloc(tmem, 256);
+    if (warp == P_WARPS) tc::dealloc(tmem, 512);
 }
 
 struct OParams {

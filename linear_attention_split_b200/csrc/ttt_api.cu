@@ -856,7 +856,9 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         pp.N = (int)N;
         pp.H = H;
         pp.d = d;
-        blk::proj_kernel<<<tiles, blk::THREADS, blk::p_smem_bytes(), st>>>(tx, tw, pp);
+        // persistent: one CTA per SM (at most), each looping over its tiles
+        blk::proj_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::THREADS, blk::p_smem_bytes(), st>>>(
+            tx, tw, pp);
         if (int rc = launched(1)) return rc;
         if (int rc = ttt_linear_fullbatch(q, k, v, w0, o, nullptr, B, H, (int)N, d, eta, dtype, core, core_bytes, stream))
             return rc;
