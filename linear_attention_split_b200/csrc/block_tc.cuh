@@ -11,8 +11,11 @@
 // output, so the core is a kernel of its own):
 //   proj : persistent, one CTA per SM looping over the 128-token tiles: x tiles through a TMA
 //          ring, Wqkvg resident (MN-major), x Wqkvg into one of two 256-column TMEM
-//          accumulators, so that the epilogue -- Q, K, V head-split [B, H, N, d] and G [B, N, C]
-//          in bf16 -- of one tile overlaps the loads and the MMAs of the next.
+//          accumulators, so that the epilogue -- Q, K, V and G token-major [B, N, C] in bf16 --
+//          of one tile overlaps the loads and the MMAs of the next.  The heads of Q, K, V sit
+//          side by side in each token's C = 64 features, the layout in which the core (the
+//          tensor-core TTT-Linear kernel) takes an image as one unit of 64 features with a
+//          block-diagonal W0.
 //   out  : per 128-token tile, four warps build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128,
 //          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows
 //          (16-byte loads, all issued up front), the conv from a window of x rows that one TMA
@@ -41,9 +44,8 @@ constexpr int O_WARPS = 16;             // out: sixteen Z / epilogue warps (row 
 constexpr int O_THREADS = 32 * O_WARPS + 32;
 
 struct PParams {
-    __nv_bfloat16 *q, *k, *v, *g;       // [B, H, N, d] x 3, [B, N, C]
+    __nv_bfloat16 *q, *k, *v, *g;       // [B, N, C] each (heads side by side in C)
     long long rows;                     // B * N
-    int N, H, d;
 };
 struct PBars {
     uint64_t wfull, xfull[PXS], xempty[PXS], done[2], tfree[2];
@@ -119,7 +121,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < nj; ++j) {
             const int b = j & 1;
             const long long R = row0_of(j) + row;
-            const long long bi = R / p.N, t = R % p.N;
             mbar_wait(&bars->done[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
             tc::fence_after();
             // this warp's 128 columns in two TMEM round trips of four 16-column chunks
@@ -139,14 +140,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const int j0 = ch * 2 * C + (4 * g4 + c4) * 16;
                     const int which = j0 / C, c = j0 % C;
-                    __nv_bfloat16* dst;
-                    if (which == 3) {
-                        dst = p.g + R * C + c;
-                    } else {
-                        const int h = c / p.d, e = c % p.d;
-                        __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : p.v;
-                        dst = base + ((bi * p.H + h) * p.N + t) * p.d + e;
-                    }
+                    __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : which == 2 ? p.v : p.g;
+                    __nv_bfloat16* dst = base + R * C + c;
                     const float* x = v[c4];
                     uint4* d4 = reinterpret_cast<uint4*>(dst);
                     d4[0] = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
@@ -164,12 +159,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 struct OParams {
     const __nv_bfloat16* x;             // [B, N, C]
-    const __nv_bfloat16* o;             // [B, H, N, d] (the core's output)
+    const __nv_bfloat16* o;             // [B, N, C] (the core's output, heads side by side)
     const __nv_bfloat16* g;             // [B, N, C]
     const float* wc;                    // [C, 3, 3]
     __nv_bfloat16* y;                   // [B, N, C]
     long long rows;
-    int N, Hg, Wg, H, d;
+    int N, Hg, Wg;
 };
 struct OBars {
     uint64_t wfull, xfull, zready, done;
@@ -247,14 +242,14 @@ __global__ void __launch_bounds__(O_THREADS, 1)
         const int row = q4 * 32 + lane;
         const long long R = row0 + row;
         const bool valid = R < p.rows;
-        const long long b = R / p.N, t = R % p.N;
+        const long long t = R % p.N;
         const int py = (int)(t / p.Wg), px = (int)(t % p.Wg);
         // the gate half's O and G rows: every load issued before any is used
         uint4 ov[2], gv[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const int c = cg * 16 + q * 8, h = c / p.d, e = c % p.d;
-            ov[q] = valid ? *reinterpret_cast<const uint4*>(p.o + ((b * p.H + h) * p.N + t) * p.d + e) : make_uint4(0, 0, 0, 0);
+            const int c = cg * 16 + q * 8;
+            ov[q] = valid ? *reinterpret_cast<const uint4*>(p.o + R * C + c) : make_uint4(0, 0, 0, 0);
             gv[q] = valid ? *reinterpret_cast<const uint4*>(p.g + R * C + c) : make_uint4(0, 0, 0, 0);
         }
         mbar_wait(&bars->xfull, 0, TTT_DEVERR_TIMEOUT_TMA);

@@ -73,9 +73,10 @@ constexpr uint32_t IDESC_WG2 = tc::idesc_bf16(128, 128, 0, 0);   // A K-major, B
 constexpr uint32_t IDESC_APPLY = tc::idesc_bf16(128, 64, 0, 0);  // A K-major (Q), B K-major (W*^T)
 
 struct Params {
-    const float* w0;    // [H][64][64]
+    const float* w0;    // [H][64][64]; with dh < 64: [64 / dh][dh][dh] (one per head of the unit)
     float* w_star;      // [U][64][64] or nullptr
     int H, N;
+    int dh;             // 64, or the width of the heads that sit side by side in a unit's 64 features
     int TT;             // token rows per tile (multiple of 16, <= 128)
     int n_tiles;        // tiles per unit, ceil(N / TT)
     int slots;          // ring slots (32 KB each)
@@ -320,7 +321,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row = q4 * 32 + lane;        // tile row / accumulator lane of this thread
         const int et = threadIdx.x - 64;       // 0..255
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-        const float* W0 = p.w0 + (size_t)(u % p.H) * D * D;
+        const float* W0 = p.dh == D ? p.w0 + (size_t)(u % p.H) * D * D : p.w0;
+        // element (m, f) of this unit's 64 x 64 W0.  With heads of dh < 64 side by side in the
+        // unit's features, W0 is block-diagonal (head h's block is w0[h]); the kernel then
+        // zeroes W*'s off-diagonal blocks, and each head's block of W* and of O is exactly its
+        // own full-batch step (G W0 and C are taken block by block).
+        auto w0at = [&](int m, int f) -> float {
+            if (p.dh == D) return __ldg(&W0[m * D + f]);
+            return (m / p.dh == f / p.dh) ? __ldg(&W0[((m / p.dh) * p.dh + m % p.dh) * p.dh + f % p.dh]) : 0.f;
+        };
 
         // ---- W0^T as bf16 hi + lo, K-major (row = output feature f, k = input feature m) --
         {
@@ -329,7 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int m = mg * 16 + 2 * k;
-                split_bf16(__ldg(&W0[m * D + f]), __ldg(&W0[(m + 1) * D + f]), hi[k], lo[k]);
+                split_bf16(w0at(m, f), w0at(m + 1, f), hi[k], lo[k]);
             }
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -350,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int it = et + k * EPI_THREADS;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                w0o[k][i] = it < items ? __ldg(&W0[(4 * (it & 15) + i) * D + r0 + (it >> 4)]) : 0.f;
+                w0o[k][i] = it < items ? w0at(4 * (it & 15) + i, r0 + (it >> 4)) : 0.f;
         }
 
         // ---- G rows of this CTA as bf16 hi + lo (a K-major operand; G is symmetric) -------
@@ -434,8 +443,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                         s.w += v.w;
                     }
                     const int f = r0 + fl;
-                    const float w[4] = {w0o[k][0] - p.eta_over_n * s.x, w0o[k][1] - p.eta_over_n * s.y,
-                                        w0o[k][2] - p.eta_over_n * s.z, w0o[k][3] - p.eta_over_n * s.w};
+                    float w[4] = {w0o[k][0] - p.eta_over_n * s.x, w0o[k][1] - p.eta_over_n * s.y,
+                                  w0o[k][2] - p.eta_over_n * s.z, w0o[k][3] - p.eta_over_n * s.w};
+                    if (p.dh < D)  // heads side by side: W* keeps only its diagonal blocks
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if ((4 * cg + i) / p.dh != f / p.dh) w[i] = 0.f;
                     if (p.w_star) {
                         float* ws = p.w_star + (size_t)u * D * D;
 #pragma unroll

@@ -218,9 +218,11 @@ int linear_tc(const void* q, const void* k, const void* v, const float* w0, void
     return launched(1);
 }
 
-// d = 64: tcgen05 kernel (one cluster of S CTAs per unit, one CTA per SM, no workspace)
+// d = 64: tcgen05 kernel (one cluster of S CTAs per unit, one CTA per SM, no workspace).
+// dh < 64: each unit's 64 features are 64 / dh heads side by side, w0 is [64 / dh][dh][dh]
+// (the block's core, whose Q, K, V are token-major [B, N, 64])
 int linear_tc5(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_star, int B, int H,
-               int N, float eta, cudaStream_t st) {
+               int N, float eta, cudaStream_t st, int dh = 64) {
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     const long long U = (long long)B * H;
@@ -243,6 +245,7 @@ int linear_tc5(const void* q, const void* k, const void* v, const float* w0, voi
     p.w_star = w_star;
     p.H = H;
     p.N = N;
+    p.dh = dh;
     p.eta_over_n = (float)((double)eta / (double)N);
     // more than half an SM's shared memory: one CTA per SM, which owns all 512 TMEM columns
     const int smem = std::max(p.slots * lin5::SLOT_BYTES + extra, dev->smem_per_sm / 2 + 1024);
@@ -853,15 +856,13 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         pp.v = static_cast<__nv_bfloat16*>(v);
         pp.g = static_cast<__nv_bfloat16*>(g);
         pp.rows = rows;
-        pp.N = (int)N;
-        pp.H = H;
-        pp.d = d;
         // persistent: one CTA per SM (at most), each looping over its tiles
         blk::proj_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::THREADS, blk::p_smem_bytes(), st>>>(
             tx, tw, pp);
         if (int rc = launched(1)) return rc;
-        if (int rc = ttt_linear_fullbatch(q, k, v, w0, o, nullptr, B, H, (int)N, d, eta, dtype, core, core_bytes, stream))
-            return rc;
+        // the core: each image is one unit of 64 features (the heads side by side, token-major),
+        // W0 block-diagonal from the heads' w0
+        if (int rc = linear_tc5(q, k, v, w0, o, nullptr, B, 1, (int)N, eta, st, d)) return rc;
         blk::OParams op;
         op.x = static_cast<const __nv_bfloat16*>(x);
         op.o = static_cast<const __nv_bfloat16*>(o);
@@ -872,8 +873,6 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         op.N = (int)N;
         op.Hg = Hg;
         op.Wg = Wg;
-        op.H = H;
-        op.d = d;
         blk::out_kernel<<<tiles, blk::O_THREADS, blk::o_smem_bytes(), st>>>(two, txw, op);
         return launched(1);
     }
