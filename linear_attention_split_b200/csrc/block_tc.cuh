@@ -56,7 +56,7 @@ constexpr int p_smem_bytes() { return PXS * XT + WQ + (int)sizeof(PBars) + 1024;
 __global__ void __launch_bounds__(THREADS, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const PParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* xs = smem_align<1024>(smem_raw);
     uint8_t* ws = xs + PXS * XT;
     PBars* bars = reinterpret_cast<PBars*>(ws + WQ);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -190,7 +190,7 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 __global__ void __launch_bounds__(O_THREADS, 1)
     out_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_xw, const OParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* zs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* zs = smem_align<1024>(smem_raw);
     uint8_t* zl = zs + ZT;                 // Z lo
     uint8_t* xw = zl + ZT;                 // x rows row0 - (Wg + 1) .. (128-byte swizzle)
     uint8_t* wos = xw + XW * ROWB;

@@ -44,6 +44,14 @@ __device__ __forceinline__ long long ttt_wait_limit() {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// The dynamic shared-memory base `raw` rounded up to ALIGN bytes.  The rounding is pointer
+// arithmetic on the __shared__ array (not a round trip through an integer), so the compiler
+// still sees a shared-memory pointer and accesses through it become shared-memory loads and
+// stores with immediate offsets instead of 64-bit generic ones.
+template <uint32_t ALIGN>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* raw) {
+    return raw + ((ALIGN - (smem_u32(raw) & (ALIGN - 1u))) & (ALIGN - 1u));
+}
 
 // ----------------------------------------------------------------------- mbarrier ----
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -173,6 +181,45 @@ __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
 }
 __device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Bounded wait with cluster-scope acquire (data written by peer CTAs with st.async).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int err) {
+    const long long limit = ttt_wait_limit();
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (ttt_timed_out()) return false;
+        if (clock64() - t0 > limit) {
+            ttt_raise(err);
+            return false;
+        }
+    }
+}
+// 16 / 8 bytes into another CTA's shared memory, completion counted on its mbarrier.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     raddr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
+                 "r"(a), "r"(b), "r"(rbar)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+    return out;
 }
 
 // ----------------------------------------------------------------------- swizzle -----

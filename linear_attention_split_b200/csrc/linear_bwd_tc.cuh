@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     reduce_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g, const RParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = smem_align<1024>(smem_raw);
     RBars* bars = reinterpret_cast<RBars*>(ring + R_STAGES * R_STAGE);
     const int S = gridDim.x, r = blockIdx.x, u = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                  const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
                  const __grid_constant__ CUtensorMap tm_dv, const AParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* ops = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ops = smem_align<1024>(smem_raw);
     uint8_t* ring = ops + OPS;
     ABars* bars = reinterpret_cast<ABars*>(ring + A_STAGES * A_STAGE);
     const int S = gridDim.x, r = blockIdx.x, u = blockIdx.y;

@@ -80,7 +80,7 @@ __global__ void __maxnreg__(200)
                      const Params p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align<1024>(smem_raw);
     const Layout<D> L(p);
     uint8_t* ring = smem + L.ring;
     uint8_t* qreg = smem + L.qreg;

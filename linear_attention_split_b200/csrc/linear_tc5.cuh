@@ -95,45 +95,6 @@ __device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 1
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Bounded wait with cluster-scope acquire (data written by peer CTAs with st.async).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int err) {
-    const long long limit = ttt_wait_limit();
-    const long long t0 = clock64();
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if (ttt_timed_out()) return false;
-        if (clock64() - t0 > limit) {
-            ttt_raise(err);
-            return false;
-        }
-    }
-}
-// 16 / 8 bytes into another CTA's shared memory, completion counted on its mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b, uint32_t c,
-                                            uint32_t d) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     raddr),
-                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
-                 : "memory");
-}
-__device__ __forceinline__ void st_async_v2(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
-                 "r"(a), "r"(b), "r"(rbar)
-                 : "memory");
-}
-__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
-    uint32_t out;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
-    return out;
-}
 // Byte offset of element (row n, column k) in a 64 x 64 bf16 K-major operand, 128-byte swizzle.
 __device__ __forceinline__ uint32_t op_off(int n, int k) {
     return (uint32_t)(n >> 3) * 1024u + swz<3>((uint32_t)(n & 7) * ROWB + (uint32_t)k * 2u);
@@ -151,7 +112,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                       const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = smem_align<1024>(smem_raw);
     uint8_t* pool = base;                                   // ring slots, then Q tiles
     uint8_t* fixed = base + p.slots * SLOT_BYTES;
     uint8_t* w0op = fixed;                                  // [W0_hi^T ; W0_lo^T] (K-major, 128 rows)

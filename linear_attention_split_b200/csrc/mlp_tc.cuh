@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     grad_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_w1,
                 const __grid_constant__ CUtensorMap tm_w2, const GradParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align<1024>(smem_raw);
     uint8_t* w1s = smem;                 // 32 KB
     uint8_t* w2s = w1s + WBYTES;         // 32 KB
     uint8_t* at = w2s + WBYTES;          // 64 KB  A = gelu(Z)
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                  const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
                  const ApplyParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align<1024>(smem_raw);
     uint8_t* w1s = smem;                 // W1* hi (bf16)
     uint8_t* w1l = w1s + WBYTES;         // W1* lo (bf16)
     uint8_t* w2s = w1l + WBYTES;         // W2* (fp16)

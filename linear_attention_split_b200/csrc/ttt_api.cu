@@ -425,21 +425,26 @@ int dwconv_fused(const void* q, const void* k, const void* v, const float* w0, v
     DeviceInfo* dev = nullptr;
     if (int rc = current_device(&dev)) return rc;
     if (B > 65535) return TTT_ERR_UNSUPPORTED;
+    // One cluster of S CTAs per image, one CTA per SM: S = 8 while the whole batch's 8-CTA
+    // clusters fit on the GPU at once (15 of them on a 148-SM B200), else 4 (33 fit); more if
+    // the rows per CTA would not fit, fewer for short grids (every CTA owns two rows or more).
     int S = 1;
-    while (S < 8 && S * 2 <= Hg) S *= 2;
+    const int s_want = B <= 15 || (Hg + 3) / 4 > dwc::MAX_R ? 8 : 4;
+    while (S < s_want && S * 2 <= Hg) S *= 2;
     dwc::Params p;
     p.R = (Hg + S - 1) / S;
     if (p.R > dwc::MAX_R) return TTT_ERR_UNSUPPORTED;
     p.cw = (Wg + dwc::PXW - 1) / dwc::PXW;
+    p.nb = 2 * p.cw <= dwc::MAX_WARPS ? 2 : 1;
     p.slot_bytes = (dwc::PXW * p.cw + 2) * dwc::PXB;
-    p.nslots = std::max(dwc::KS + dwc::VS, p.R + 2);
+    p.nslots = std::max(p.nb * (dwc::KS + dwc::VS), p.R + 2);
     p.w0 = w0;
     p.w_star = w_star;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.Hg = Hg;
     p.Wg = Wg;
     p.eta_over_n = (float)((double)eta / ((double)Hg * Wg));
-    const int smem = p.nslots * p.slot_bytes + (2 + dwc::MAX_CW) * dwc::C * dwc::NTAP * 4 + (int)sizeof(dwc::Bars) + 128;
+    const int smem = p.nslots * p.slot_bytes + (2 + dwc::MAX_WARPS) * dwc::C * dwc::NTAP * 4 + (int)sizeof(dwc::Bars) + 128;
     if (smem > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
     CUtensorMap tk, tv, tq;
     if (!tmap_bf16_rows(&tk, k, dwc::C, Wg, Hg, B) || !tmap_bf16_rows(&tv, v, dwc::C, Wg, Hg, B) ||
@@ -451,7 +456,7 @@ int dwconv_fused(const void* q, const void* k, const void* v, const float* w0, v
         return TTT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(S, (unsigned)B, 1);
-    cfg.blockDim = dim3((p.cw + 1) * 32, 1, 1);
+    cfg.blockDim = dim3((p.nb * p.cw + 1) * 32, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -38,6 +38,14 @@ def test_dwconv_grids(Hg, Wg):
     check_dwconv(2, Hg, Wg, 64, "bf16", seed=Hg * 100 + Wg)
 
 
+@pytest.mark.parametrize("B,Hg,Wg", [(3, 56, 56), (2, 64, 64), (2, 20, 84), (1, 150, 12), (40, 8, 8), (2, 9, 90)])
+def test_dwconv_c64_shapes(B, Hg, Wg):
+    """C = 64 bf16 shapes around the fused kernel's limits: an odd batch, the widest fused grid
+    (eight strips, one band), more clusters than fit at once (two waves), and grids past the
+    fused kernel (wider than 64 tokens, more than 16 rows per CTA: general kernel)."""
+    check_dwconv(B, Hg, Wg, 64, "bf16", seed=B * 1000 + Hg + Wg)
+
+
 @pytest.mark.parametrize("C", [8, 24, 3])
 def test_dwconv_channels(C):
     check_dwconv(3, 10, 12, C, "bf16")
