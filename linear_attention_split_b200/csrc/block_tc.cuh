@@ -16,12 +16,15 @@
 //          side by side in each token's C = 64 features, the layout in which the core (the
 //          tensor-core TTT-Linear kernel) takes an image as one unit of 64 features with a
 //          block-diagonal W0.
-//   out  : per 128-token tile, four warps build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128,
-//          fp32, kept as bf16 hi + lo, K-major) in shared memory -- the gate from O and G rows
-//          (16-byte loads, all issued up front), the conv from a window of x rows that one TMA
-//          box brings in (the tile's rows and one grid row plus one token on each side, at most
-//          256 rows, so Wg <= 63) -- then one MMA chain Z_hi Wo + Z_lo Wo (K = 128, N = 64) and
-//          the epilogue stores y in bf16.
+//   out  : persistent, one CTA per SM looping over the 128-token tiles.  Per tile sixteen warps
+//          build Z = [O * sigmoid(G) | dwconv3x3(x)] (128 x 128, fp32, kept as bf16 hi + lo,
+//          K-major) in shared memory -- the gate from O and G rows (16-byte loads, issued one
+//          tile ahead into registers), the conv from a window of x rows that one TMA box brings
+//          in (the tile's rows and one grid row plus one token on each side, at most 256 rows,
+//          so Wg <= 63) -- then one MMA chain Z_hi Wo + Z_lo Wo (K = 128, N = 64) and the
+//          epilogue stores y in bf16.  Two x windows, two Z buffers and two TMEM accumulators:
+//          while the tensor cores project tile i, the warps build tile i + 1 and the producer
+//          brings tile i + 2's window.
 // No token-tile output is written twice and no intermediate of the out kernel (Z) goes to HBM.
 #pragma once
 #include "common.cuh"
@@ -167,10 +170,10 @@ struct OParams {
     int N, Hg, Wg;
 };
 struct OBars {
-    uint64_t wfull, xfull, zready, done;
+    uint64_t wfull, xfull[2], xempty[2], zready[2], done[2], tfree[2];
     uint32_t tmem_base;
 };
-constexpr int o_smem_bytes() { return 2 * ZT + XW * ROWB + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
+constexpr int o_smem_bytes() { return 4 * ZT + 2 * XW * ROWB + WO + C * 9 * 4 + (int)sizeof(OBars) + 1024; }
 
 // 1 / (1 + e^-z) with the fast exponential and the fast (approximate, ~2 ulp) division
 __device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
@@ -190,19 +193,25 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 __global__ void __launch_bounds__(O_THREADS, 1)
     out_kernel(const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_xw, const OParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* zs = smem_align<1024>(smem_raw);
-    uint8_t* zl = zs + ZT;                 // Z lo
-    uint8_t* xw = zl + ZT;                 // x rows row0 - (Wg + 1) .. (128-byte swizzle)
-    uint8_t* wos = xw + XW * ROWB;
+    uint8_t* base = smem_align<1024>(smem_raw);
+    auto zbuf = [&](int b) { return base + b * 2 * ZT; };              // Z hi, then Z lo
+    auto xwin = [&](int b) { return base + 4 * ZT + b * XW * ROWB; };  // x rows around a tile (128-byte swizzle)
+    uint8_t* wos = base + 4 * ZT + 2 * XW * ROWB;
     float* wcs = reinterpret_cast<float*>(wos + WO);
     OBars* bars = reinterpret_cast<OBars*>(wcs + C * 9);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row0 = (long long)blockIdx.x * MT;
+    const long long ntiles = (p.rows + MT - 1) / MT;
+    const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA
+    auto tile_of = [&](int j) { return (long long)blockIdx.x + (long long)j * gridDim.x; };
     if (threadIdx.x == 32 * O_WARPS) {
         mbar_init(&bars->wfull, 1);
-        mbar_init(&bars->xfull, 1);
-        mbar_init(&bars->zready, O_WARPS);
-        mbar_init(&bars->done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->xfull[b], 1);
+            mbar_init(&bars->xempty[b], O_WARPS);
+            mbar_init(&bars->zready[b], O_WARPS);
+            mbar_init(&bars->done[b], 1);
+            mbar_init(&bars->tfree[b], O_WARPS);
+        }
         mbar_fence_init();
     }
     // taps regrouped as [8-channel chunk][tap][8 channels]: one tap of a chunk is two float4
@@ -210,122 +219,163 @@ __global__ void __launch_bounds__(O_THREADS, 1)
         const int ch = e / 9, tap = e % 9;
         wcs[((ch >> 3) * 9 + tap) * 8 + (ch & 7)] = p.wc[e];
     }
-    if (warp == O_WARPS) tc::alloc(&bars->tmem_base, 64);
+    if (warp == O_WARPS) tc::alloc(&bars->tmem_base, 128);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars->tmem_base;
     if (warp == O_WARPS) {
+        // ======================= producer of the x windows and MMA issuer =========================
         if (lane == 0) {
-            mbar_expect_tx(&bars->xfull, XW * ROWB);  // rows outside the tensor are zero-filled
-            tma_load_3d(xw, &tm_xw, 0, (int)(row0 - (p.Wg + 1)), 0, &bars->xfull);
+            auto load_x = [&](int j) {  // the window of this CTA's j-th tile into buffer j & 1
+                const int b = j & 1;
+                if (j >= 2) mbar_wait(&bars->xempty[b], ((j >> 1) - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                mbar_expect_tx(&bars->xfull[b], XW * ROWB);  // rows outside the tensor are zero-filled
+                tma_load_3d(xwin(b), &tm_xw, 0, (int)(tile_of(j) * MT - (p.Wg + 1)), 0, &bars->xfull[b]);
+            };
             mbar_expect_tx(&bars->wfull, WO);
             tma_load_3d(wos, &tm_wo, 0, 0, 0, &bars->wfull);
+            for (int j = 0; j < 2 && j < nj; ++j) load_x(j);
             mbar_wait(&bars->wfull, 0, TTT_DEVERR_TIMEOUT_TMA);
-            mbar_wait(&bars->zready, 0, TTT_DEVERR_TIMEOUT_PEER);
-            tc::fence_after();
             const uint32_t wa = smem_u32(wos);
             constexpr uint32_t ID = tc::idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
+            for (int j = 0; j < nj; ++j) {
+                const int b = j & 1;
+                mbar_wait(&bars->zready[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                if (j >= 2) mbar_wait(&bars->tfree[b], ((j >> 1) - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+                tc::fence_after();
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl) {
-                const uint32_t za = smem_u32(hl ? zl : zs);
+                for (int hl = 0; hl < 2; ++hl) {
+                    const uint32_t za = smem_u32(zbuf(b) + hl * ZT);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_bf16(tmem, tc::smem_desc(za + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
-                                 tc::smem_desc(wa + ks * 2048, 8192, 1024, 2), ID, (hl > 0 || ks > 0) ? 1 : 0);
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc::mma_bf16(tmem + b * 64, tc::smem_desc(za + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2),
+                                     tc::smem_desc(wa + ks * 2048, 8192, 1024, 2), ID, (hl > 0 || ks > 0) ? 1 : 0);
+                }
+                tc::commit(&bars->done[b]);
+                if (j + 2 < nj) load_x(j + 2);  // this tile's window has been read (zready)
             }
-            tc::commit(&bars->done);
         }
     } else {
+        // ======================= Z builders and epilogue (sixteen warps) ==========================
         // warp w: token rows of lane quarter w % 4, channels 16 (w / 4) .. + 15 (two 8-channel chunks)
         const int q4 = warp & 3, cg = warp >> 2;
         const int row = q4 * 32 + lane;
-        const long long R = row0 + row;
-        const bool valid = R < p.rows;
-        const long long t = R % p.N;
-        const int py = (int)(t / p.Wg), px = (int)(t % p.Wg);
-        // the gate half's O and G rows: every load issued before any is used
-        uint4 ov[2], gv[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int c = cg * 16 + q * 8;
-            ov[q] = valid ? *reinterpret_cast<const uint4*>(p.o + R * C + c) : make_uint4(0, 0, 0, 0);
-            gv[q] = valid ? *reinterpret_cast<const uint4*>(p.g + R * C + c) : make_uint4(0, 0, 0, 0);
-        }
-        mbar_wait(&bars->xfull, 0, TTT_DEVERR_TIMEOUT_TMA);
-        const int wrow = row + p.Wg + 1;  // this token's row in the x window
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int c = cg * 16 + q * 8, chunk = c >> 3;
-            uint4 mz = make_uint4(0, 0, 0, 0), dz = mz, mzl = mz, dzl = mz;
-            if (valid) {
-                const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[q]);
-                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[q]);
-                float m[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 of = __bfloat1622float2(o2[i]), gf = __bfloat1622float2(g2[i]);
-                    m[2 * i] = of.x * sigmoidf_(gf.x);
-                    m[2 * i + 1] = of.y * sigmoidf_(gf.y);
-                }
-                split8(m, mz, mzl);
-                uint64_t acc2[4] = {0, 0, 0, 0};  // channel pairs (2i, 2i + 1), packed fp32
-#pragma unroll
-                for (int a = 0; a < 3; ++a)
-#pragma unroll
-                    for (int bb = 0; bb < 3; ++bb) {
-                        const int yy = py + a - 1, xx = px + bb - 1;
-                        if (yy < 0 || yy >= p.Hg || xx < 0 || xx >= p.Wg) continue;
-                        const int wr = wrow + (a - 1) * p.Wg + (bb - 1);  // same image: inside the window
-                        const uint4 raw = *reinterpret_cast<const uint4*>(xw + wr * ROWB + ((chunk ^ (wr & 7)) << 4));
-                        const float4* wt = reinterpret_cast<const float4*>(wcs + (chunk * 9 + a * 3 + bb) * 8);
-                        const float4 w0 = wt[0], w1 = wt[1];
-                        const uint64_t wp[4] = {
-                            (uint64_t)__float_as_uint(w0.x) | ((uint64_t)__float_as_uint(w0.y) << 32),
-                            (uint64_t)__float_as_uint(w0.z) | ((uint64_t)__float_as_uint(w0.w) << 32),
-                            (uint64_t)__float_as_uint(w1.x) | ((uint64_t)__float_as_uint(w1.y) << 32),
-                            (uint64_t)__float_as_uint(w1.z) | ((uint64_t)__float_as_uint(w1.w) << 32)};
-                        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {  // bf16 pair -> fp32 pair, then one fma per lane
-                            const uint64_t f = (uint64_t)(rw[i] << 16) | ((uint64_t)(rw[i] & 0xffff0000u) << 32);
-                            asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2[i]) : "l"(wp[i]), "l"(f));
-                        }
-                    }
-                float acc[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc[2 * i] = __uint_as_float((uint32_t)acc2[i]);
-                    acc[2 * i + 1] = __uint_as_float((uint32_t)(acc2[i] >> 32));
-                }
-                split8(acc, dz, dzl);
-            }
-            const uint32_t off = swz<3>((uint32_t)row * ROWB + c * 2);
-            *reinterpret_cast<uint4*>(zs + off) = mz;
-            *reinterpret_cast<uint4*>(zs + 16384 + off) = dz;
-            *reinterpret_cast<uint4*>(zl + off) = mzl;
-            *reinterpret_cast<uint4*>(zl + 16384 + off) = dzl;
-        }
-        fence_proxy_async_smem();  // read next by the tensor cores
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->zready);
-        mbar_wait(&bars->done, 0, TTT_DEVERR_TIMEOUT_TMA);
-        tc::fence_after();
-        // y: this warp's 16 output columns of its lane quarter
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-        float v[16];
-        tc::ld16(lane_base + cg * 16, v);
-        tc::wait_ld();
-        if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(p.y + R * C + cg * 16);
-            d4[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-            d4[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
-                               pack_bf16(v[14], v[15]));
+        // the gate half's O and G rows of tile j (two 8-channel chunks each)
+        struct OG {
+            uint4 o[2], g[2];
+        };
+        auto load_og = [&](int j) {
+            OG r;
+            const long long R = tile_of(j) * MT + row;
+            const bool valid = R < p.rows;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int c = cg * 16 + q * 8;
+                r.o[q] = valid ? *reinterpret_cast<const uint4*>(p.o + R * C + c) : make_uint4(0, 0, 0, 0);
+                r.g[q] = valid ? *reinterpret_cast<const uint4*>(p.g + R * C + c) : make_uint4(0, 0, 0, 0);
+            }
+            return r;
+        };
+        auto epilogue = [&](int j) {  // y of tile j from its TMEM accumulator
+            const int b = j & 1;
+            mbar_wait(&bars->done[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+            tc::fence_after();
+            float v[16];
+            tc::ld16(lane_base + b * 64 + cg * 16, v);
+            tc::wait_ld();
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tfree[b]);
+            const long long R = tile_of(j) * MT + row;
+            if (R < p.rows) {
+                uint4* d4 = reinterpret_cast<uint4*>(p.y + R * C + cg * 16);
+                d4[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                   pack_bf16(v[6], v[7]));
+                d4[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                                   pack_bf16(v[14], v[15]));
+            }
+        };
+        OG cur = load_og(0);  // nj >= 1: the grid has at most one CTA per tile
+        for (int j = 0; j < nj; ++j) {
+            const int b = j & 1;
+            const OG nxt = load_og(j + 1 < nj ? j + 1 : j);  // next tile's rows, requested before this tile's work
+            const long long R = tile_of(j) * MT + row;
+            const bool valid = R < p.rows;
+            const long long t = valid ? R % p.N : 0;
+            const int py = (int)(t / p.Wg), px = (int)(t % p.Wg);
+            // Z buffer b was last read by tile j - 2's MMAs, which this warp's epilogue of tile
+            // j - 2 (previous iteration) waited for
+            mbar_wait(&bars->xfull[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+            const uint8_t* xw = xwin(b);
+            uint8_t* zs = zbuf(b);
+            uint8_t* zl = zs + ZT;
+            const int wrow = row + p.Wg + 1;  // this token's row in the x window
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int c = cg * 16 + q * 8, chunk = c >> 3;
+                uint4 mz = make_uint4(0, 0, 0, 0), dz = mz, mzl = mz, dzl = mz;
+                if (valid) {
+                    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&cur.o[q]);
+                    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&cur.g[q]);
+                    float m[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 of = __bfloat1622float2(o2[i]), gf = __bfloat1622float2(g2[i]);
+                        m[2 * i] = of.x * sigmoidf_(gf.x);
+                        m[2 * i + 1] = of.y * sigmoidf_(gf.y);
+                    }
+                    split8(m, mz, mzl);
+                    float2 acc2[4] = {};  // channel pairs (2i, 2i + 1)
+#pragma unroll
+                    for (int a = 0; a < 3; ++a)
+#pragma unroll
+                        for (int bb = 0; bb < 3; ++bb) {
+                            const int yy = py + a - 1, xx = px + bb - 1;
+                            if (yy < 0 || yy >= p.Hg || xx < 0 || xx >= p.Wg) continue;
+                            const int wr = wrow + (a - 1) * p.Wg + (bb - 1);  // same image: inside the window
+                            const uint4 raw = *reinterpret_cast<const uint4*>(xw + wr * ROWB + ((chunk ^ (wr & 7)) << 4));
+                            const float4* wt = reinterpret_cast<const float4*>(wcs + (chunk * 9 + a * 3 + bb) * 8);
+                            const float4 w0 = wt[0], w1 = wt[1];
+                            const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                                                  make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
+                            const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)  // bf16 pair -> fp32 pair, then one packed fma
+                                acc2[i] = __ffma2_rn(wp[i],
+                                                     make_float2(__uint_as_float(rw[i] << 16),
+                                                                 __uint_as_float(rw[i] & 0xffff0000u)),
+                                                     acc2[i]);
+                        }
+                    float acc[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] = acc2[i].x;
+                        acc[2 * i + 1] = acc2[i].y;
+                    }
+                    split8(acc, dz, dzl);
+                }
+                const uint32_t off = swz<3>((uint32_t)row * ROWB + c * 2);
+                *reinterpret_cast<uint4*>(zs + off) = mz;
+                *reinterpret_cast<uint4*>(zs + 16384 + off) = dz;
+                *reinterpret_cast<uint4*>(zl + off) = mzl;
+                *reinterpret_cast<uint4*>(zl + 16384 + off) = dzl;
+            }
+            fence_proxy_async_smem();  // read next by the tensor cores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->xempty[b]);  // the window may take tile j + 2's rows
+                mbar_arrive(&bars->zready[b]);
+            }
+            if (j >= 1) epilogue(j - 1);
+            cur = nxt;
         }
+        epilogue(nj - 1);
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == O_WARPS) tc::dealloc(tmem, 64);
+    if (warp == O_WARPS) tc::dealloc(tmem, 128);
 }
 
 }  // namespace blk

@@ -878,7 +878,9 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         op.N = (int)N;
         op.Hg = Hg;
         op.Wg = Wg;
-        blk::out_kernel<<<tiles, blk::O_THREADS, blk::o_smem_bytes(), st>>>(two, txw, op);
+        // persistent: one CTA per SM (at most), each looping over its tiles
+        blk::out_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::O_THREADS, blk::o_smem_bytes(), st>>>(
+            two, txw, op);
         return launched(1);
     }
     float* z = reinterpret_cast<float*>(static_cast<char*>(core) + core_bytes);
