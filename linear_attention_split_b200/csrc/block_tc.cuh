@@ -11,8 +11,9 @@
 // output, so the core is a kernel of its own):
 //   proj : persistent, one CTA per SM looping over the 128-token tiles: x tiles through a TMA
 //          ring, Wqkvg resident (MN-major), x Wqkvg into one of two 256-column TMEM
-//          accumulators, so that the epilogue -- Q, K, V and G token-major [B, N, C] in bf16 --
-//          of one tile overlaps the loads and the MMAs of the next.  The heads of Q, K, V sit
+//          accumulators, so that the epilogue -- Q, K, V and G token-major [B, N, C] in bf16,
+//          staged per tile in shared memory (128-byte swizzle) and written by one TMA store
+//          per tensor -- of one tile overlaps the loads and the MMAs of the next.  The heads of Q, K, V sit
 //          side by side in each token's C = 64 features, the layout in which the core (the
 //          tensor-core TTT-Linear kernel) takes an image as one unit of 64 features with a
 //          block-diagonal W0.
@@ -47,21 +48,23 @@ constexpr int O_WARPS = 16;             // out: sixteen Z / epilogue warps (row 
 constexpr int O_THREADS = 32 * O_WARPS + 32;
 
 struct PParams {
-    __nv_bfloat16 *q, *k, *v, *g;       // [B, N, C] each (heads side by side in C)
-    long long rows;                     // B * N
+    long long rows;                     // B * N (Q, K, V, G [B, N, C] each, heads side by side in C)
 };
 struct PBars {
     uint64_t wfull, xfull[PXS], xempty[PXS], done[2], tfree[2];
     uint32_t tmem_base;
 };
-constexpr int p_smem_bytes() { return PXS * XT + WQ + (int)sizeof(PBars) + 1024; }
+constexpr int p_smem_bytes() { return PXS * XT + WQ + 4 * XT + (int)sizeof(PBars) + 1024; }
 
 __global__ void __launch_bounds__(THREADS, 1)
-    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const PParams p) {
+    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g, const PParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* xs = smem_align<1024>(smem_raw);
     uint8_t* ws = xs + PXS * XT;
-    PBars* bars = reinterpret_cast<PBars*>(ws + WQ);
+    uint8_t* st = ws + WQ;  // the tile's Q, K, V, G (16 KB each, 128-byte swizzle) for the TMA stores
+    PBars* bars = reinterpret_cast<PBars*>(st + 4 * XT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long ntiles = (p.rows + MT - 1) / MT;
     const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA (>= 1)
@@ -121,11 +124,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q4 = warp & 3, ch = warp >> 2;  // lane quarter, column half (Q, K | V, G)
         const int row = q4 * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+        const CUtensorMap* maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
+        const bool storer = threadIdx.x == 0;
         for (int j = 0; j < nj; ++j) {
             const int b = j & 1;
-            const long long R = row0_of(j) + row;
             mbar_wait(&bars->done[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
             tc::fence_after();
+            // the previous tile's stores have read the staging buffers
+            if (storer) tma_store_wait_read_all();
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * P_WARPS) : "memory");
             // this warp's 128 columns in two TMEM round trips of four 16-column chunks
 #pragma unroll 1
             for (int g4 = 0; g4 < 2; ++g4) {
@@ -138,22 +145,30 @@ __global__ void __launch_bounds__(THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->tfree[b]);
                 }
-                if (R >= p.rows) continue;
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const int j0 = ch * 2 * C + (4 * g4 + c4) * 16;
                     const int which = j0 / C, c = j0 % C;
-                    __nv_bfloat16* base = which == 0 ? p.q : which == 1 ? p.k : which == 2 ? p.v : p.g;
-                    __nv_bfloat16* dst = base + R * C + c;
                     const float* x = v[c4];
-                    uint4* d4 = reinterpret_cast<uint4*>(dst);
-                    d4[0] = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                                       pack_bf16(x[6], x[7]));
-                    d4[1] = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]),
-                                       pack_bf16(x[14], x[15]));
+                    uint8_t* tile = st + which * XT + row * ROWB;
+                    const int k0 = c / 8;  // 16-byte chunk of the 128-byte row
+                    *reinterpret_cast<uint4*>(tile + ((k0 ^ (row & 7)) << 4)) =
+                        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                   pack_bf16(x[6], x[7]));
+                    *reinterpret_cast<uint4*>(tile + (((k0 + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]),
+                                   pack_bf16(x[14], x[15]));
                 }
             }
+            fence_proxy_async_smem();  // read next by the TMA stores
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * P_WARPS) : "memory");
+            if (storer) {  // rows past the tensor are clipped by the hardware
+#pragma unroll
+                for (int w = 0; w < 4; ++w) tma_store_3d(maps[w], 0, (int)row0_of(j), 0, st + w * XT);
+                tma_store_commit();
+            }
         }
+        if (storer) tma_store_wait_all();
     }
     tc::fence_before();
     __syncthreads();

@@ -843,8 +843,10 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         if (blk::p_smem_bytes() > dev->smem_optin || blk::o_smem_bytes() > dev->smem_optin) return TTT_ERR_UNSUPPORTED;
         if ((rows + blk::MT - 1) / blk::MT > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
         const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-        CUtensorMap tx, tw, two, txw;
+        CUtensorMap tx, tw, two, txw, tq, tk, tv, tg;
         if (!tmap_bf16_3d(&tx, x, blk::C, (int)rows, 1, blk::MT, sw) ||
+            !tmap_bf16_3d(&tq, q, blk::C, (int)rows, 1, blk::MT, sw) || !tmap_bf16_3d(&tk, k, blk::C, (int)rows, 1, blk::MT, sw) ||
+            !tmap_bf16_3d(&tv, v, blk::C, (int)rows, 1, blk::MT, sw) || !tmap_bf16_3d(&tg, g, blk::C, (int)rows, 1, blk::MT, sw) ||
             !tmap_bf16_3d(&txw, x, blk::C, (int)rows, 1, blk::XW, sw) ||
             !tmap_bf16_box(&tw, wqkvg, 4 * blk::C, blk::C, 1, 64, 64, sw) ||
             !tmap_bf16_box(&two, wo, blk::C, 2 * blk::C, 1, 64, 2 * blk::C, sw))
@@ -856,14 +858,10 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
             return TTT_ERR_CUDA;
         const unsigned tiles = (unsigned)((rows + blk::MT - 1) / blk::MT);
         blk::PParams pp;
-        pp.q = static_cast<__nv_bfloat16*>(q);
-        pp.k = static_cast<__nv_bfloat16*>(k);
-        pp.v = static_cast<__nv_bfloat16*>(v);
-        pp.g = static_cast<__nv_bfloat16*>(g);
         pp.rows = rows;
         // persistent: one CTA per SM (at most), each looping over its tiles
         blk::proj_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::THREADS, blk::p_smem_bytes(), st>>>(
-            tx, tw, pp);
+            tx, tw, tq, tk, tv, tg, pp);
         if (int rc = launched(1)) return rc;
         // the core: each image is one unit of 64 features (the heads side by side, token-major),
         // W0 block-diagonal from the heads' w0
