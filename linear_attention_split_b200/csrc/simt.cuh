@@ -438,12 +438,19 @@ __global__ void __launch_bounds__(TPB) linear_bwd_apply(const T* __restrict__ k,
 __global__ void __launch_bounds__(TPB) linear_bwd_dw0(const float* __restrict__ dw0u, float* __restrict__ dw0, int B,
                                                       int H, int d) {
     const int h = blockIdx.x;
-    const int e = blockIdx.y * TPB + threadIdx.x;
+    const int e = blockIdx.y * blockDim.x + threadIdx.x;
     const int dd = d * d;
     if (e >= dd) return;
     float s = 0.f;
-#pragma unroll 8
-    for (int b = 0; b < B; ++b) s += dw0u[((long long)b * H + h) * dd + e];  // batch order
+    int b = 0;
+    for (; b + 16 <= B; b += 16) {  // sixteen loads in flight, then the adds in batch order
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = dw0u[((long long)(b + i) * H + h) * dd + e];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s += x[i];
+    }
+    for (; b < B; ++b) s += dw0u[((long long)b * H + h) * dd + e];
     dw0[(long long)h * dd + e] = s;
 }
 

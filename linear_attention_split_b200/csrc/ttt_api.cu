@@ -356,8 +356,8 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     ap.n_tiles = pl.n_tiles;
     lbw::apply_kernel<<<dim3(pl.S, (unsigned)U), lbw::A_THREADS, lbw::a_smem_bytes(), st>>>(tops, tg, tk, tv, tdq,
                                                                                              tdk, tdv, ap);
-    simt::linear_bwd_dw0<<<dim3((unsigned)H, (lbw::DD + simt::TPB - 1) / simt::TPB), simt::TPB, 0, st>>>(dw0u, dw0, B,
-                                                                                                       H, lbw::D);
+    // the batch sum of dW0: 64-thread blocks, so that the 4096 elements spread over 64 SMs
+    simt::linear_bwd_dw0<<<dim3((unsigned)H, (lbw::DD + 63) / 64), 64, 0, st>>>(dw0u, dw0, B, H, lbw::D);
     return launched(4);
 }
 
