@@ -12,8 +12,9 @@
 //   proj : persistent, one CTA per SM looping over the 128-token tiles: x tiles through a TMA
 //          ring, Wqkvg resident (MN-major), x Wqkvg into one of two 256-column TMEM
 //          accumulators, so that the epilogue -- Q, K, V and G token-major [B, N, C] in bf16,
-//          staged per tile in shared memory (128-byte swizzle) and written by one TMA store
-//          per tensor -- of one tile overlaps the loads and the MMAs of the next.  The heads of Q, K, V sit
+//          staged per tile in one of two shared-memory buffers (128-byte swizzle) and written
+//          by one TMA store per tensor -- of one tile overlaps the loads and the MMAs of the
+//          next, and its stores drain while the next tile is staged.  The heads of Q, K, V sit
 //          side by side in each token's C = 64 features, the layout in which the core (the
 //          tensor-core TTT-Linear kernel) takes an image as one unit of 64 features with a
 //          block-diagonal W0.
@@ -54,7 +55,7 @@ struct PBars {
     uint64_t wfull, xfull[PXS], xempty[PXS], done[2], tfree[2];
     uint32_t tmem_base;
 };
-constexpr int p_smem_bytes() { return PXS * XT + WQ + 4 * XT + (int)sizeof(PBars) + 1024; }
+constexpr int p_smem_bytes() { return PXS * XT + WQ + 8 * XT + (int)sizeof(PBars) + 1024; }
 
 __global__ void __launch_bounds__(THREADS, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -63,8 +64,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* xs = smem_align<1024>(smem_raw);
     uint8_t* ws = xs + PXS * XT;
-    uint8_t* st = ws + WQ;  // the tile's Q, K, V, G (16 KB each, 128-byte swizzle) for the TMA stores
-    PBars* bars = reinterpret_cast<PBars*>(st + 4 * XT);
+    uint8_t* st = ws + WQ;  // two buffers of a tile's Q, K, V, G (16 KB each, 128-byte swizzle) for the TMA stores
+    PBars* bars = reinterpret_cast<PBars*>(st + 8 * XT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long ntiles = (p.rows + MT - 1) / MT;
     const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA (>= 1)
@@ -130,8 +131,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int b = j & 1;
             mbar_wait(&bars->done[b], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
             tc::fence_after();
-            // the previous tile's stores have read the staging buffers
-            if (storer) tma_store_wait_read_all();
+            // the stores of tile j - 2 (this staging buffer) have read it; tile j - 1's may go on
+            uint8_t* stj = st + (j & 1) * 4 * XT;
+            if (storer) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
             asm volatile("bar.sync 1, %0;" ::"n"(32 * P_WARPS) : "memory");
             // this warp's 128 columns in two TMEM round trips of four 16-column chunks
 #pragma unroll 1
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int j0 = ch * 2 * C + (4 * g4 + c4) * 16;
                     const int which = j0 / C, c = j0 % C;
                     const float* x = v[c4];
-                    uint8_t* tile = st + which * XT + row * ROWB;
+                    uint8_t* tile = stj + which * XT + row * ROWB;
                     const int k0 = c / 8;  // 16-byte chunk of the 128-byte row
                     *reinterpret_cast<uint4*>(tile + ((k0 ^ (row & 7)) << 4)) =
                         make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("bar.sync 1, %0;" ::"n"(32 * P_WARPS) : "memory");
             if (storer) {  // rows past the tensor are clipped by the hardware
 #pragma unroll
-                for (int w = 0; w < 4; ++w) tma_store_3d(maps[w], 0, (int)row0_of(j), 0, st + w * XT);
+                for (int w = 0; w < 4; ++w) tma_store_3d(maps[w], 0, (int)row0_of(j), 0, stj + w * XT);
                 tma_store_commit();
             }
         }
