@@ -608,16 +608,25 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(&bars->oread[ob]);
             // both column halves of every row quarter are in shared memory once oread completes
             mbar_wait(&bars->oread[ob], (j >> 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
-            if (ch == 0 && lane == 0) {
-                const int row0 = j * MT + q4 * 32;
-                if (row0 < n_valid) {
-                    tma_store_3d(&tm_o, 0, t0 + row0, u, tile + q4 * 32 * ROWB);
-                    tma_store_commit();
-                    tma_store_wait_read_all();
+            if (ch == 0) {
+                // the row quarter's store; this warp releases the Q buffer of tile j - 1 once that
+                // tile's store has read it, so no store is waited for on the way to the next gelu
+                if (lane == 0) {
+                    const int row0 = j * MT + q4 * 32;
+                    if (row0 < n_valid) {
+                        tma_store_3d(&tm_o, 0, t0 + row0, u, tile + q4 * 32 * ROWB);
+                        tma_store_commit();
+                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                    } else {
+                        tma_store_wait_read_all();
+                    }
                 }
+                __syncwarp();
+                if (lane == 0 && j >= 1) mbar_arrive(&bars->qfree[(j - 1) % NQB]);
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->qfree[b]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->qfree[b]);
         };
         // gelu of tile i, then the output of tile i - 1 (whose MMAs ran meanwhile)
         for (int i = 0; i < ntiles; ++i) {
@@ -645,6 +654,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (ntiles > 0) o_store(ntiles - 1);
         if (lane == 0) tma_store_wait_all();
+        __syncwarp();
+        if (ch == 0 && lane == 0 && ntiles > 0) mbar_arrive(&bars->qfree[(ntiles - 1) % NQB]);
     }
     tc::fence_before();
     __syncthreads();
