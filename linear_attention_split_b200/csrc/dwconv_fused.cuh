@@ -8,9 +8,11 @@
 //     g[t]    = (1/N) sum_p r(p) K(p + off_t)          (N = Hg * Wg)
 //     w*[c]   = w0[c] - eta g
 //     O(p)    = sum_t w*[c][t] Q(p + off_t)
-// Design (B200): one thread-block cluster of S CTAs per image, one CTA per SM (so every CTA of
-// a cluster runs at the same pace), CTA r owning output rows [r*R, r*R + R).  The CTA's rows
-// form NB bands (two when the width allows fourteen consumer warps) that advance side by side.
+// Design (B200): one thread-block cluster of S CTAs per image, CTA r owning output rows
+// [r*R, r*R + R).  The CTA's rows form NB bands (two when the width allows fourteen consumer
+// warps) that advance side by side; at a 56-token width that is fifteen warps and one CTA per
+// SM, so every CTA of a cluster runs at the same pace (with two CTAs per SM, some SMs held
+// one and the clusters waited for their SM-sharing CTAs).
 // A producer warp streams each band's K rows (with the one-row halo above and below,
 // zero-filled by TMA outside the image) and V rows through small TMA rings; the consumer
 // warps of a band each own a strip of pixels, each lane a pair of channels, and keep the
