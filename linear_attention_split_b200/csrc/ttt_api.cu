@@ -22,6 +22,7 @@
 #include "linear_bwd_tc.cuh"
 #include "block_tc.cuh"
 #include "dwconv_fused.cuh"
+#include "apply_tc.cuh"
 #include "chunked_tc.cuh"
 #include "mlp_tc.cuh"
 
@@ -1043,6 +1044,21 @@ size_t ttt_linear_minibatch_workspace_bytes(int B, int H, int N, int d, int chun
     return own;
 }
 
+// O = Q W per unit for a given fp32 W [U][64][64], bf16 Q and O [U][N][64]: the tensor-core output pass.
+int apply_w_tc(const void* q, const float* w, void* out, long long U, int N, cudaStream_t st) {
+    if (U > 65535) return TTT_ERR_UNSUPPORTED;
+    CUtensorMap tq, to;
+    if (!tmap_bf16_3d(&tq, q, atc::D, N, (int)U, atc::MT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tmap_bf16_3d(&to, out, atc::D, N, (int)U, atc::MT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TTT_ERR_CUDA;
+    if (cudaFuncSetAttribute(atc::apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, atc::smem_bytes()) !=
+        cudaSuccess)
+        return TTT_ERR_CUDA;
+    atc::apply_kernel<<<dim3((unsigned)((N + atc::MT - 1) / atc::MT), (unsigned)U), atc::THREADS, atc::smem_bytes(),
+                        st>>>(tq, to, w);
+    return launched(1);
+}
+
 int ttt_linear_minibatch(const void* q, const void* k, const void* v, const float* w0, void* out, float* w_final,
                          int B, int H, int N, int d, int chunk, int epochs, float eta, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
@@ -1069,10 +1085,7 @@ int ttt_linear_minibatch(const void* q, const void* k, const void* v, const floa
     const float eta_over_b = (float)((double)eta / (double)chunk);
     if (chunked_tc_ok(B, H, d, chunk, dtype)) {  // the tensor-core recurrence in training mode
         if (int rc = chunked_tc(q, k, v, w0, out, B, H, N, eta, 1, nullptr, st, epochs, wfin, w_final)) return rc;
-        using T = __nv_bfloat16;
-        simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(static_cast<const T*>(q), wfin,
-                                                                                    static_cast<T*>(out), N, d);
-        return launched(1);
+        return apply_w_tc(q, wfin, out, U, N, st);
     }
     if (dtype == TTT_BF16) {
         using T = __nv_bfloat16;
