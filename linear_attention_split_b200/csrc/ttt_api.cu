@@ -1094,6 +1094,10 @@ int ttt_linear_minibatch(const void* q, const void* k, const void* v, const floa
             return TTT_ERR_CUDA;
         simt::minibatch_train<T><<<(unsigned)U, simt::TPB, smem, st>>>(
             static_cast<const T*>(k), static_cast<const T*>(v), w0, wfin, w_final, H, N, d, chunk, epochs, eta_over_b);
+        if (d == atc::D) {  // the output pass on the tensor cores
+            if (int rc = launched(1)) return rc;
+            return apply_w_tc(q, wfin, out, U, N, st);
+        }
         simt::linear_apply<T><<<grid_units(U, (long long)N * d), simt::TPB, 0, st>>>(static_cast<const T*>(q), wfin,
                                                                                     static_cast<T*>(out), N, d);
     } else {

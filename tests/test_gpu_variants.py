@@ -57,6 +57,7 @@ def test_one_way_scans_sum_to_bidirectional_on_gpu():
     (2, 2, 3136, 64, 64, 1, "bf16"),     # mini-batches of 64, one epoch
     (2, 2, 1024, 64, 64, 2, "bf16"),     # two epochs
     (8, 1, 3136, 64, 64, 2, "bf16"),     # the benchmarked 56x56 shape: 49 chunks x 2 epochs
+    (2, 3, 1000, 64, 40, 2, "bf16"),     # chunks of 40 (CUDA-core training), tensor-core output pass, ragged tile
     (2, 1, 196, 64, 196, 3, "f32"),      # full batch, three epochs
     (1, 2, 96, 32, 16, 2, "f32"),
 ])
