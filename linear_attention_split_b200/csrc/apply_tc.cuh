@@ -60,14 +60,23 @@ __global__ void __launch_bounds__(THREADS)
     }
     // W (row k = input feature, column n = output feature) -> operand row n, column k, as
     // bf16 hi + lo; consecutive threads take consecutive n, so the reads of W are coalesced
+    // (all of a thread's loads are issued before any is used: one L2 round trip)
     const float* wu = w + (size_t)u * D * D;
-    for (int e = threadIdx.x; e < D * D / 2; e += THREADS) {
-        const int n = e % D, kp = e / D;
-        const float a = __ldg(wu + (2 * kp) * D + n), b = __ldg(wu + (2 * kp + 1) * D + n);
-        const uint32_t hi = pack_bf16(a, b);
+    constexpr int PER = D * D / 2 / THREADS;  // input-row pairs per thread
+    float wa[PER], wb[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = threadIdx.x + i * THREADS, n = e % D, kp = e / D;
+        wa[i] = __ldg(wu + (2 * kp) * D + n);
+        wb[i] = __ldg(wu + (2 * kp + 1) * D + n);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = threadIdx.x + i * THREADS, n = e % D, kp = e / D;
+        const uint32_t hi = pack_bf16(wa[i], wb[i]);
         const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xffff0000u);
         *reinterpret_cast<uint32_t*>(wh + op_off(n, 2 * kp)) = hi;
-        *reinterpret_cast<uint32_t*>(wl + op_off(n, 2 * kp)) = pack_bf16(a - ha, b - hb);
+        *reinterpret_cast<uint32_t*>(wl + op_off(n, 2 * kp)) = pack_bf16(wa[i] - ha, wb[i] - hb);
     }
     fence_proxy_async_smem();  // read next by the tensor cores
     tc::fence_before();
