@@ -149,6 +149,12 @@ __device__ __forceinline__ void tma_store_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// ----------------------------------------------------------------------- grid dependency ---
+// Programmatic dependent launch: wait until the previous grid on the stream has completed (and
+// its writes are visible); let the next grid's CTAs start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------------- clusters ----
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

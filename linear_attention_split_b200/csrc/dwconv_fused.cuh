@@ -145,6 +145,18 @@ __global__ void __maxnreg__(128)
     fence_proxy_async_smem();
     __syncthreads();
     cluster_arrive_release();  // this CTA's barriers are initialised (waited on before any st.async)
+    // Launched with programmatic stream serialization: the first K and V rows go into L2 while the
+    // previous grid on the stream may still run (a prefetch only warms the coherent L2); every
+    // load and store of this grid comes after griddep_wait.
+    if (threadIdx.x == 32 * NW && rows > 0)
+        for (int n = 0; n < NB; ++n)
+            for (int k = 0; k < min(KS, rows_of(n) + 2); ++k) {
+                const int y = y0 + n * band_rows - 1 + k;
+                if (y >= 0 && y < p.Hg) tma_prefetch_l2_4d(&tm_k, 0, 0, y, b);
+                if (k < min(VS, rows_of(n)) && y + 1 < p.Hg) tma_prefetch_l2_4d(&tm_v, 0, 0, y + 1, b);
+            }
+    griddep_wait();
+    griddep_launch();  // one wave: the next grid's CTAs start only as SMs free up
 
     if (warp == NW) {
         // ================================ producer ======================================

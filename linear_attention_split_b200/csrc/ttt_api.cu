@@ -460,13 +460,17 @@ int dwconv_fused(const void* q, const void* k, const void* v, const float* w0, v
     cfg.blockDim = dim3((p.nb * p.cw + 1) * 32, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the kernel waits for the previous grid (griddepcontrol.wait)
+    // before its first global memory access
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, p) != cudaSuccess) return TTT_ERR_CUDA;
     return launched(1);
 }
