@@ -70,6 +70,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long ntiles = (p.rows + MT - 1) / MT;
     const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA (>= 1)
     auto row0_of = [&](int j) { return ((long long)blockIdx.x + (long long)j * gridDim.x) * MT; };
+    // Launched with programmatic stream serialization: the first x tiles go into L2 while the
+    // previous grid on the stream may still run (a prefetch only warms the coherent L2); every
+    // load and store of this grid comes after griddep_wait.
+    if (threadIdx.x == 32 * (P_WARPS + 1))
+        for (int j = 0; j < min(PXS, nj); ++j) tma_prefetch_l2_3d(&tm_x, 0, (int)row0_of(j), 0);
+    griddep_wait();
+    griddep_launch();
     if (threadIdx.x == 32 * P_WARPS) {
         mbar_init(&bars->wfull, 1);
         for (int s = 0; s < PXS; ++s) {
@@ -220,6 +227,13 @@ __global__ void __launch_bounds__(O_THREADS, 1)
     const long long ntiles = (p.rows + MT - 1) / MT;
     const int nj = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);  // tiles of this CTA
     auto tile_of = [&](int j) { return (long long)blockIdx.x + (long long)j * gridDim.x; };
+    // Launched with programmatic stream serialization: the first two x windows go into L2 while
+    // the previous grid (the core) may still run; every load and store comes after griddep_wait.
+    if (threadIdx.x == 32 * O_WARPS)
+        for (int j = 0; j < 2 && j < nj; ++j)
+            tma_prefetch_l2_3d(&tm_xw, 0, (int)max(0LL, tile_of(j) * MT - (p.Wg + 1)), 0);
+    griddep_wait();
+    griddep_launch();
     if (threadIdx.x == 32 * O_WARPS) {
         mbar_init(&bars->wfull, 1);
         for (int b = 0; b < 2; ++b) {

@@ -865,8 +865,19 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         blk::PParams pp;
         pp.rows = rows;
         // persistent: one CTA per SM (at most), each looping over its tiles
-        blk::proj_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::THREADS, blk::p_smem_bytes(), st>>>(
-            tx, tw, tq, tk, tv, tg, pp);
+        // programmatic dependent launch (proj and out): each kernel waits for the previous grid
+        // (griddepcontrol.wait) before its first global memory access
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3(std::min<unsigned>(tiles, (unsigned)dev->sms), 1, 1);
+        pc.blockDim = dim3(blk::THREADS, 1, 1);
+        pc.dynamicSmemBytes = blk::p_smem_bytes();
+        pc.stream = st;
+        pc.attrs = pdl;
+        pc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&pc, blk::proj_kernel, tx, tw, tq, tk, tv, tg, pp) != cudaSuccess) return TTT_ERR_CUDA;
         if (int rc = launched(1)) return rc;
         // the core: each image is one unit of 64 features (the heads side by side, token-major),
         // W0 block-diagonal from the heads' w0
@@ -882,8 +893,10 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
         op.Hg = Hg;
         op.Wg = Wg;
         // persistent: one CTA per SM (at most), each looping over its tiles
-        blk::out_kernel<<<std::min<unsigned>(tiles, (unsigned)dev->sms), blk::O_THREADS, blk::o_smem_bytes(), st>>>(
-            two, txw, op);
+        cudaLaunchConfig_t oc = pc;
+        oc.blockDim = dim3(blk::O_THREADS, 1, 1);
+        oc.dynamicSmemBytes = blk::o_smem_bytes();
+        if (cudaLaunchKernelEx(&oc, blk::out_kernel, two, txw, op) != cudaSuccess) return TTT_ERR_CUDA;
         return launched(1);
     }
     float* z = reinterpret_cast<float*>(static_cast<char*>(core) + core_bytes);
