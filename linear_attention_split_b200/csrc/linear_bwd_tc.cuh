@@ -61,6 +61,19 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int TT = p.TT;
     const int n_t = r < p.n_tiles ? (p.n_tiles - r + S - 1) / S : 0;
+    // Launched with programmatic stream serialization: the first tiles go into L2 while the
+    // previous grid on the stream may still run (a prefetch only warms the coherent L2); every
+    // load and store of this grid comes after griddep_wait.
+    if (threadIdx.x == 0)
+        for (int i = 0; i < min(R_STAGES, n_t); ++i) {
+            const int row = (r + i * S) * TT;
+            tma_prefetch_l2_3d(&tm_v, 0, row, u);
+            tma_prefetch_l2_3d(&tm_k, 0, row, u);
+            tma_prefetch_l2_3d(&tm_q, 0, row, u);
+            tma_prefetch_l2_3d(&tm_g, 0, row, u);
+        }
+    griddep_wait();
+    griddep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < R_STAGES; ++s) {
             mbar_init(&bars->full[s], 1);
@@ -238,6 +251,8 @@ __global__ void __launch_bounds__(256) finish_kernel(const FParams p) {
     float* Aop = fsm;                 // [k][row]
     float* Bop = fsm + D * FLD;       // [k][col]
     const int u = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+    griddep_wait();  // the partials of the reduce grid
+    griddep_launch();
     const float* W0 = p.w0 + (size_t)(u % p.H) * DD;
     const float* part = p.part + (size_t)u * p.S * 3 * DD;
     // operands: j = 0: A[k][r] = G[k][r] (= G[r][k]: G = K^T K from exact bf16 products is
@@ -379,6 +394,16 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int TT = p.TT;
     const int n_t = r < p.n_tiles ? (p.n_tiles - r + S - 1) / S : 0;
+    // the first dO, K, V tiles (inputs of the call) into L2 before waiting for the finish grid
+    if (threadIdx.x == 0)
+        for (int i = 0; i < min(A_STAGES, n_t); ++i) {
+            const int row = (r + i * S) * TT;
+            tma_prefetch_l2_3d(&tm_g, 0, row, u);
+            tma_prefetch_l2_3d(&tm_k, 0, row, u);
+            tma_prefetch_l2_3d(&tm_v, 0, row, u);
+        }
+    griddep_wait();
+    griddep_launch();
     if (threadIdx.x == 0) {
         mbar_init(&bars->opfull, 1);
         for (int s = 0; s < A_STAGES; ++s) {

@@ -440,6 +440,7 @@ __global__ void __launch_bounds__(TPB) linear_bwd_dw0(const float* __restrict__ 
     const int h = blockIdx.x;
     const int e = blockIdx.y * blockDim.x + threadIdx.x;
     const int dd = d * d;
+    griddep_wait();  // under programmatic dependent launch: the per-unit dW0 of the previous grid
     if (e >= dd) return;
     float s = 0.f;
     int b = 0;

@@ -342,7 +342,24 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     rp.part = part;
     rp.TT = pl.TT;
     rp.n_tiles = pl.n_tiles;
-    lbw::reduce_kernel<<<dim3(pl.S, (unsigned)U), lbw::R_THREADS, lbw::r_smem_bytes(), st>>>(tv, tk, tq, tg, rp);
+    // the four launches use programmatic dependent launch: each kernel requests its first input
+    // tiles into L2 (where they are inputs of the call) and then waits for the previous grid
+    // (griddepcontrol.wait) before its first global memory access
+    auto pdl = [&](auto kern, dim3 grid, int threads, int smem, auto... args) -> int {
+        cudaLaunchConfig_t c = {};
+        c.gridDim = grid;
+        c.blockDim = dim3((unsigned)threads, 1, 1);
+        c.dynamicSmemBytes = (size_t)smem;
+        c.stream = st;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        a[0].val.programmaticStreamSerializationAllowed = 1;
+        c.attrs = a;
+        c.numAttrs = 1;
+        return cudaLaunchKernelEx(&c, kern, args...) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+    };
+    if (int rc = pdl(lbw::reduce_kernel, dim3(pl.S, (unsigned)U), lbw::R_THREADS, lbw::r_smem_bytes(), tv, tk, tq, tg, rp))
+        return rc;
     lbw::FParams fp;
     fp.part = part;
     fp.w0 = w0;
@@ -351,14 +368,17 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     fp.H = H;
     fp.S = pl.S;
     fp.eta_over_n = (float)((double)eta / (double)N);
-    lbw::finish_kernel<<<dim3((unsigned)U, 3), 256, lbw::f_smem_bytes(), st>>>(fp);
+    if (int rc = pdl(lbw::finish_kernel, dim3((unsigned)U, 3), 256, lbw::f_smem_bytes(), fp)) return rc;
     lbw::AParams ap;
     ap.TT = pl.TT;
     ap.n_tiles = pl.n_tiles;
-    lbw::apply_kernel<<<dim3(pl.S, (unsigned)U), lbw::A_THREADS, lbw::a_smem_bytes(), st>>>(tops, tg, tk, tv, tdq,
-                                                                                             tdk, tdv, ap);
+    if (int rc = pdl(lbw::apply_kernel, dim3(pl.S, (unsigned)U), lbw::A_THREADS, lbw::a_smem_bytes(), tops, tg, tk, tv,
+                     tdq, tdk, tdv, ap))
+        return rc;
     // the batch sum of dW0: 64-thread blocks, so that the 4096 elements spread over 64 SMs
-    simt::linear_bwd_dw0<<<dim3((unsigned)H, (lbw::DD + 63) / 64), 64, 0, st>>>(dw0u, dw0, B, H, lbw::D);
+    if (int rc = pdl(simt::linear_bwd_dw0, dim3((unsigned)H, (lbw::DD + 63) / 64), 64, 0, (const float*)dw0u, dw0, B, H,
+                     lbw::D))
+        return rc;
     return launched(4);
 }
 
