@@ -307,6 +307,23 @@ size_t bwd_simt_ws(long long U, int d) {
     return align256((size_t)U * 3 * d * d * 4) + align256((size_t)U * 2 * d * d * 4) + align256((size_t)U * d * d * 4);
 }
 
+// Launch with programmatic dependent launch: the kernel may start while the previous grid on the
+// stream finishes and waits for it (griddepcontrol.wait) before its first global memory access.
+template <typename Kern, typename... Args>
+int launch_pdl(Kern kern, dim3 grid, int threads, int smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = grid;
+    c.blockDim = dim3((unsigned)threads, 1, 1);
+    c.dynamicSmemBytes = (size_t)smem;
+    c.stream = st;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
+    c.attrs = a;
+    c.numAttrs = 1;
+    return cudaLaunchKernelEx(&c, kern, args...) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
 int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, const void* g, void* dq, void* dk,
                   void* dv, float* dw0, int B, int H, int N, float eta, void* ws, cudaStream_t st) {
     DeviceInfo* dev = nullptr;
@@ -344,19 +361,8 @@ int linear_bwd_tc(const void* q, const void* k, const void* v, const float* w0, 
     rp.n_tiles = pl.n_tiles;
     // the four launches use programmatic dependent launch: each kernel requests its first input
     // tiles into L2 (where they are inputs of the call) and then waits for the previous grid
-    // (griddepcontrol.wait) before its first global memory access
-    auto pdl = [&](auto kern, dim3 grid, int threads, int smem, auto... args) -> int {
-        cudaLaunchConfig_t c = {};
-        c.gridDim = grid;
-        c.blockDim = dim3((unsigned)threads, 1, 1);
-        c.dynamicSmemBytes = (size_t)smem;
-        c.stream = st;
-        cudaLaunchAttribute a[1];
-        a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        a[0].val.programmaticStreamSerializationAllowed = 1;
-        c.attrs = a;
-        c.numAttrs = 1;
-        return cudaLaunchKernelEx(&c, kern, args...) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+    auto pdl = [&](auto kern, dim3 grid, int threads, int smem, auto... args) {
+        return launch_pdl(kern, grid, threads, smem, st, args...);
     };
     if (int rc = pdl(lbw::reduce_kernel, dim3(pl.S, (unsigned)U), lbw::R_THREADS, lbw::r_smem_bytes(), tv, tk, tq, tg, rp))
         return rc;
