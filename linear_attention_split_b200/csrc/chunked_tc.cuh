@@ -126,11 +126,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_v16);
+            // every wait of this kernel leaves out the suspend-time hint: the chain of chunk
+            // steps hands off through barriers, and the hardware's own limit wakes it sooner
             for (int step = 0; step < steps; ++step)
                 for (int dir = 0; dir < 2; ++dir) {
                     if (!active(dir)) continue;
                     const int s = step % STAGES, use = step / STAGES;
-                    if (use > 0) mbar_wait(&bars->empty[dir][s], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                    if (use > 0) mbar_wait<false>(&bars->empty[dir][s], (use - 1) & 1, TTT_DEVERR_TIMEOUT_TMA);
                     const int t0 = chunk_of(dir, step) * CB;
                     uint8_t* dst = stage_ptr(dir, s);
                     mbar_expect_tx(&bars->full[dir][s], train ? STAGE - TILE : STAGE);
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 16 ks..): registers {0, 2} / {1, 3} are the B fragments of K_i^T for tokens
         // 16 i + 0..7 / 16 i + 8..15.
         uint32_t ka[4][4][4];
-        mbar_wait(&bars->full[dir][0], 0, TTT_DEVERR_TIMEOUT_TMA);
+        mbar_wait<false>(&bars->full[dir][0], 0, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(&bars->empty[dir][s]);  // K, V of this step consumed
             // the next step's K fragments load while this step's dW drains
             if (step + 1 < steps) {
-                if (!nf) mbar_wait(&bars->full[dir][sn], ((step + 1) / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
+                if (!nf) mbar_wait<false>(&bars->full[dir][sn], ((step + 1) / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             make_a();
             if (train) continue;  // training mode: no output per chunk
             // ---- hand W (after this step, fp32) to the output warp ---------------------------
-            if (!wf) mbar_wait(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
+            if (!wf) mbar_wait<false>(&bars->wfree[dir][b], (use - 1) & 1, TTT_DEVERR_TIMEOUT_PEER);
             {
                 float4* dst = reinterpret_cast<float4*>(wfr_ptr(dir, b));
 #pragma unroll
@@ -327,12 +329,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int step = 0; step < nc; ++step) {
         const int s = step % STAGES;
         const int b = step % WBUF, use = step / WBUF;
-        mbar_wait(&bars->full[dir][s], (step / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
+        mbar_wait<false>(&bars->full[dir][s], (step / STAGES) & 1, TTT_DEVERR_TIMEOUT_TMA);
         const uint32_t qb = smem_u32(stage_ptr(dir, s)) + TILE;
         uint32_t qa[4][4];
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) load_a(qb, OUT_TILES * hf, ks, qa[ks]);
-        mbar_wait(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
+        mbar_wait<false>(&bars->wready[dir][b], use & 1, TTT_DEVERR_TIMEOUT_PEER);
         // B fragments of W as bf16 hi + lo: k-step ks, column tile j (the recurrence warp's
         // W^T accumulator pairs, packed as its A fragments are)
         uint32_t bw[2][4][2][2];
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (step >= a0) {
             // second visit: add the partner's partial, round once, store O.  Every read of the
             // slot is issued before the first store, so that no read waits behind a store.
-            mbar_wait(&bars->pfull[dir][hf][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1,
+            mbar_wait<false>(&bars->pfull[dir][hf][(step - a0) % (PF + 1)], ((step - a0) / (PF + 1)) & 1,
                       TTT_DEVERR_TIMEOUT_TMA);
             const float* other = reinterpret_cast<const float*>(pk + ((step - a0) % (PF + 1)) * PKB);
             float2 x[OUT_TILES][2][2];

@@ -69,21 +69,35 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// The waiting thread is suspended (it issues nothing) until the phase completes or, at the
-// latest, TTT_WAIT_SUSPEND_NS have passed; waiting warps then leave the issue slots to the
-// warps that have work.
+// With SUSPEND the waiting thread is suspended (it issues nothing) until the phase completes
+// or, at the latest, TTT_WAIT_SUSPEND_NS have passed, so waiting warps leave the issue slots to
+// the warps that have work.  Without it the wait uses the hardware's own time limit.  Measured
+// on B200, per kernel: the suspend hint is faster where many warps wait while a few compute
+// (TTT-Linear full batch 13.84 against 14.09 us, the ViT^3 block, the backward), the hardware
+// limit where a latency-bound chain hands off through barriers (the chunked scan 92.7 against
+// 94.2 us).
 #ifndef TTT_WAIT_SUSPEND_NS
 #define TTT_WAIT_SUSPEND_NS 1000000u
 #endif
+template <bool SUSPEND = true>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(TTT_WAIT_SUSPEND_NS)
-        : "memory");
+    if constexpr (SUSPEND)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(TTT_WAIT_SUSPEND_NS)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 // Non-blocking test of a phase (for polling several barriers in turn).
@@ -100,11 +114,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait: returns false (and raises `err`) if the phase does not complete within the
 // wait limit, and at once if another wait on this device has already run out.
+template <bool SUSPEND = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int err) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<SUSPEND>(bar, parity)) return true;
     const long long limit = ttt_wait_limit();
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait<SUSPEND>(bar, parity)) {
         if (ttt_timed_out()) return false;
         if (clock64() - t0 > limit) {
             ttt_raise(err);
