@@ -417,7 +417,10 @@ def run_ours(args):
         "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "peak_source": ("measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                                     if peak_src == "measured" else
+                                     f"fallback: {FALLBACK_HBM_GBS:.0f} GB/s, an earlier B200 copy "
+                                     "measurement (MEASURED_PEAKS.json absent)"),
                      "kernel": "lin5::linear_tc5_kernel", "kernel_source_sha": sha,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor_tflops": alg_flops / (ms_step / 1e3) / 1e12},
@@ -428,7 +431,7 @@ def run_ours(args):
 
     if not args.no_extras:
         rec["e2e"] = e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, min(args.steps, 200), world, pg)
-        rec["other_paths"] = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust)
+        rec["other_paths"] = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, peak_src=peak_src)
         if rank == 0 and world == 1:
             rec["cpu_baseline"] = cpu_oracle_rate(args.cpu_seconds, B, H, N, d)
             rec["cpu_baseline"]["configs"] = cpu_config_rates()
@@ -497,7 +500,7 @@ def e2e_leg(ttt, dev, stream, w0, B, H, N, d, eta, steps, world, pg):
                     "buffer sets with copy-in, compute and copy-out streams (both PCIe directions busy)"}
 
 
-def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=None):
+def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=None, peak_src=None):
     """Device time per call of the other paths at their workload shapes.  Each path cycles
     through rotating input/output sets whose total exceeds four times the L2 (so inputs come
     from HBM), K calls in one CUDA graph, timed like the headline.  `only` restricts the run
@@ -552,8 +555,8 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=
         res["mlp_64x64_d64_h256"] = {"ms": ms, "tokens_per_s": 16 * 4096 / (ms / 1e3), "tflops": tf,
                                      "frac_of_tensor_peak": tf / tf_burst,
                                      "frac_of_sustained_peak": tf / tf_sust,
-                                     "peak": "burst bf16 (MEASURED_PEAKS.json bf16_tflops): 10 calls, "
-                                             "a few ms in all"}
+                                     "peak": "burst bf16 (MEASURED_PEAKS.json bf16_tflops, else the "
+                                             "fallback in res['peaks']): 10 calls, a few ms in all"}
         del S, ws
     if only in (None, "chunked"):  # chunked bidirectional, B=8, H=3, N=6400, d=64, chunk 64
         nb = 8 * 8 * 3 * 6400 * 64
@@ -640,6 +643,8 @@ def other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=None, iters=
                                           "kernels_per_call": 3}
         del S, ws
     assert ttt.device_error() == 0
+    res["peaks"] = {"hbm_gbs": hbm_peak, "bf16_tflops_burst": tf_burst,
+                    "bf16_tflops_sustained": tf_sust, "source": peak_src}
     return res
 
 
@@ -649,9 +654,10 @@ def run_only(args):
     from linear_attention_split_b200 import ttt
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    hbm_peak, tf_burst, tf_sust, _ = peaks()
+    hbm_peak, tf_burst, tf_sust, peak_src = peaks()
     stream = torch.cuda.Stream(device=dev)
-    res = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=args.only, iters=args.steps)
+    res = other_paths(ttt, dev, stream, hbm_peak, tf_burst, tf_sust, only=args.only, iters=args.steps,
+                      peak_src=peak_src)
     print(json.dumps({"only": args.only, "steps": args.steps, "result": res}), flush=True)
 
 
