@@ -95,3 +95,33 @@ def test_chunked_conv_shapes(Hg, Wg, d, chunk, dtype):
     ro = oracle.linear_chunked_prep(inp["q"], inp["k"], inp["v"], inp["w0"], inp["wk"], inp["wv"], Hg, Wg, chunk,
                                     eta=0.7)
     assert_close(out, ro, inp["q"].dtype, f"conv scan {Hg}x{Wg} d={d} b={chunk} {dtype}", rounding_floor="auto")
+
+
+# ============================================================== determinism ===========
+def test_minibatch_deterministic_full_shape():
+    """Training-mode scan and the output pass: two calls give bit-identical O and W_final at
+    the benchmarked shape (B=32 images of 56x56, b = 64, two epochs)."""
+    g = cuda(inputs.linear_inputs(32, 1, 3136, 64, dtype="bf16", seed=6))
+    o1, w1 = ttt.linear_minibatch(g["q"], g["k"], g["v"], g["w0"], 64, 2, with_w_final=True)
+    o2, w2 = ttt.linear_minibatch(g["q"], g["k"], g["v"], g["w0"], 64, 2, with_w_final=True)
+    assert ttt.device_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(w1, w2)
+
+
+@pytest.mark.parametrize("direction", [1, -1])
+def test_one_way_deterministic_full_shape(direction):
+    g = cuda(inputs.chunked_inputs(8, 3, 6400, 64, dtype="bf16", seed=6))
+    o1 = ttt.linear_chunked(g["q"], g["k"], g["v"], g["w0"], 64, direction=direction)
+    o2 = ttt.linear_chunked(g["q"], g["k"], g["v"], g["w0"], 64, direction=direction)
+    assert ttt.device_error() == 0
+    assert torch.equal(o1, o2)
+
+
+def test_chunked_conv_deterministic_full_shape():
+    """Preprocessing pass + bidirectional scan at the benchmarked shape (B=8, 3 heads, 80x80)."""
+    g = cuda(inputs.chunked_conv_inputs(8, 3, 80, 80, 64, dtype="bf16", seed=6))
+    args = (g["q"], g["k"], g["v"], g["w0"], g["wk"], g["wv"], 80, 80, 64)
+    o1 = ttt.linear_chunked_conv(*args)
+    o2 = ttt.linear_chunked_conv(*args)
+    assert ttt.device_error() == 0
+    assert torch.equal(o1, o2)
