@@ -20,7 +20,8 @@
  *     caller's next synchronisation.
  *   - `workspace` is caller-owned device scratch of at least the size the matching
  *     *_workspace_bytes() query returns for the same arguments (it may be NULL when that
- *     size is 0).  The library allocates no device memory and keeps no per-call state.
+ *     size is 0), 16-byte aligned like the tensors (a misaligned one is TTT_ERR_INVALID_ARG).
+ *     The library allocates no device memory and keeps no per-call state.
  *   - Arguments are checked on the host before anything is enqueued.  Return codes:
  *       TTT_OK, TTT_ERR_INVALID_ARG (null pointer, size <= 0, misalignment, non-finite eta,
  *       inconsistent shape), TTT_ERR_UNSUPPORTED (a size outside the supported range),

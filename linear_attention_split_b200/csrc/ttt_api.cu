@@ -824,6 +824,7 @@ int ttt_linear_fullbatch(const void* q, const void* k, const void* v, const floa
     if (d > 128) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_linear_fullbatch_workspace_bytes(B, H, N, d, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == TTT_BF16) {
         if (d == 64) return linear_tc5(q, k, v, w0, out, w_star, B, H, N, eta, st);
@@ -859,6 +860,7 @@ int ttt_vit3_block(const void* x, const void* wqkvg, const float* w0, const floa
     if (N > 0x7fffffffLL || C / H > 128 || C > 1024) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_vit3_block_workspace_bytes(B, Hg, Wg, C, H, dtype);
     if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const long long rows = (long long)B * N;
     const int d = C / H;
@@ -983,6 +985,7 @@ int ttt_linear_fullbatch_bwd(const void* q, const void* k, const void* v, const 
     if (d > 128) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_linear_fullbatch_bwd_workspace_bytes(B, H, N, d, dtype);
     if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (linear_bwd_tc_ok(d, dtype))
         return linear_bwd_tc(q, k, v, w0, dout, dq, dk, dv, dw0, B, H, N, eta, workspace, st);
@@ -1007,6 +1010,7 @@ int ttt_dwconv_fullbatch(const void* q, const void* k, const void* v, const floa
     if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return TTT_ERR_INVALID_ARG;
     const size_t need = ttt_dwconv_fullbatch_workspace_bytes(B, Hg, Wg, C, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dwconv_fused_ok(Hg, Wg, C, dtype)) return dwconv_fused(q, k, v, w0, out, w_star, B, Hg, Wg, eta, st);
     if (dtype == TTT_BF16)
@@ -1032,6 +1036,7 @@ int ttt_mlp_fullbatch(const void* q, const void* k, const void* v, const float* 
     if (d > 256 || hidden > 4096) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_mlp_fullbatch_workspace_bytes(B, H, N, d, hidden, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (mlp_tc_ok(B, H, d, hidden, dtype))
         return mlp_tc(q, k, v, w1, w2, out, w1_star, w2_star, B, H, N, eta, workspace, st);
@@ -1059,6 +1064,7 @@ int ttt_linear_chunked(const void* q, const void* k, const void* v, const float*
     if (d > 128) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_linear_chunked_workspace_bytes(B, H, N, d, chunk, direction, dtype);
     if (workspace_bytes < need || (need && !workspace)) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (chunked_tc_ok(B, H, d, chunk, dtype))
         return chunked_tc(q, k, v, w0, out, B, H, N, eta, direction, need ? workspace : nullptr, st);
@@ -1113,6 +1119,7 @@ int ttt_linear_minibatch(const void* q, const void* k, const void* v, const floa
     if (d > 128) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_linear_minibatch_workspace_bytes(B, H, N, d, chunk, epochs, dtype);
     if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     // one epoch over one chunk of all N tokens is the full-batch step
     if (chunk == N && epochs == 1)
         return ttt_linear_fullbatch(q, k, v, w0, out, w_final, B, H, N, d, eta, dtype, workspace, workspace_bytes,
@@ -1179,6 +1186,7 @@ int ttt_linear_chunked_conv(const void* q, const void* k, const void* v, const f
     if (d > 128) return TTT_ERR_UNSUPPORTED;
     const size_t need = ttt_linear_chunked_conv_workspace_bytes(B, H, Hg, Wg, d, chunk, direction, dtype);
     if (workspace_bytes < need || !workspace) return TTT_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TTT_ERR_INVALID_ARG;
     const long long U = (long long)B * H;
     if (!grid_ok(U, N * d)) return TTT_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

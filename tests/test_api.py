@@ -203,3 +203,26 @@ def test_block_rejects_bad_arguments(L):
     a[14] = 64
     assert f(*a) == 3
     assert L.ttt_vit3_block_workspace_bytes(2, 8, 8, 64, 2, 1) >= 5 * 2 * 64 * 64 * 2
+
+
+def test_misaligned_workspace_is_rejected(L):
+    """The workspace, like every tensor, must be 16-byte aligned: a misaligned one is refused on
+    the host (TTT_ERR_INVALID_ARG) instead of reaching a TMA or bulk copy on the device."""
+    big = 1 << 30
+    assert lin(L, dt=0, ws=MISALIGNED, wsb=big) == 1
+    assert L.ttt_dwconv_fullbatch(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 4, 8, 1.0, 1, MISALIGNED, big,
+                                  None) == 1
+    assert L.ttt_mlp_fullbatch(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 64, 64, 256, 1.0, 1,
+                               MISALIGNED, big, None) == 1
+    assert L.ttt_linear_chunked_bidir(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 64, 1.0, 1, MISALIGNED, big,
+                                      None) == 1
+    assert L.ttt_linear_chunked(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 64, 1.0, -1, 1, MISALIGNED, big,
+                                None) == 1
+    assert L.ttt_linear_minibatch(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 64, 2, 1.0, 1, MISALIGNED,
+                                  big, None) == 1
+    assert L.ttt_linear_chunked_conv(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 8, 64, 64, 1.0, 0, 1,
+                                     MISALIGNED, big, None) == 1
+    assert L.ttt_linear_fullbatch_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1, 128, 64, 1.0, 1,
+                                      MISALIGNED, big, None) == 1
+    assert L.ttt_vit3_block(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 8, 64, 2, 1.0, 1, MISALIGNED, big,
+                            None) == 1
