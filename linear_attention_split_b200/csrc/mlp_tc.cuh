@@ -440,33 +440,61 @@ struct UpdateParams {
 // Block (u, c): rows h in [64 c, 64 c + 64) of gW1^T and gW2.  The S partials are added in
 // split order (deterministic).  W2*[h][d] is written row by row; W1*[d][h] is the transpose of
 // the gW1^T block, so that block goes through shared memory and leaves row by row as well.
+// Each thread takes four consecutive columns (one float4 chunk of the swizzled partials), so
+// every load is 16 bytes and every store 8 or 16.
 __global__ void __launch_bounds__(256) update_kernel(const UpdateParams p) {
     __shared__ float tile[64][65];  // W1*^T block: [h - h0][d]
     const int u = blockIdx.x, hd = u % p.H, h0 = blockIdx.y * 64;
     const float* part = p.part + (size_t)u * p.S * 2 * HID * D;
-    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 columns x 4 rows per pass
-    for (int rr = ty; rr < 64; rr += 4) {
+    const int c = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 chunks of 4 columns x 16 rows per pass
+    for (int rr = ty; rr < 64; rr += 16) {
         const int h = h0 + rr;
-        // element (h, d = tx): float4 chunk (tx / 4) ^ (h & 7) of row h in a partial
-        const int pe = h * D + ((((tx >> 2) ^ (h & 7))) << 2) + (tx & 3);
-        float g1 = 0.f, g2 = 0.f;
+        // columns d = 4 c .. 4 c + 3 of row h: float4 chunk c ^ (h & 7) of that row in a partial
+        const int pe = h * D + ((c ^ (h & 7)) << 2);
+        float g1[4] = {0.f, 0.f, 0.f, 0.f}, g2[4] = {0.f, 0.f, 0.f, 0.f};
         for (int sp = 0; sp < p.S; ++sp) {  // split order
-            g1 += part[(size_t)sp * 2 * HID * D + pe];
-            g2 += part[(size_t)sp * 2 * HID * D + HID * D + pe];
+            const float4 a = *reinterpret_cast<const float4*>(part + (size_t)sp * 2 * HID * D + pe);
+            const float4 b = *reinterpret_cast<const float4*>(part + (size_t)sp * 2 * HID * D + HID * D + pe);
+            g1[0] += a.x;
+            g1[1] += a.y;
+            g1[2] += a.z;
+            g1[3] += a.w;
+            g2[0] += b.x;
+            g2[1] += b.y;
+            g2[2] += b.z;
+            g2[3] += b.w;
         }
-        const float w2 = p.w2[(size_t)hd * HID * D + h * D + tx] - p.eta_over_n * g2;  // W2*[h][d]
-        if (p.w2_star) p.w2_star[(size_t)u * HID * D + h * D + tx] = w2;
-        p.w2h[(size_t)u * HID * D + h * D + tx] = __float2half_rn(w2);
-        tile[rr][tx] = g1;  // gW1^T[h][d]
+        const size_t o2 = (size_t)h * D + 4 * c;
+        const float4 w2o = *reinterpret_cast<const float4*>(p.w2 + (size_t)hd * HID * D + o2);
+        const float w2[4] = {w2o.x - p.eta_over_n * g2[0], w2o.y - p.eta_over_n * g2[1],
+                             w2o.z - p.eta_over_n * g2[2], w2o.w - p.eta_over_n * g2[3]};  // W2*[h][d]
+        if (p.w2_star)
+            *reinterpret_cast<float4*>(p.w2_star + (size_t)u * HID * D + o2) = make_float4(w2[0], w2[1], w2[2], w2[3]);
+        const __half2 f01 = __floats2half2_rn(w2[0], w2[1]), f23 = __floats2half2_rn(w2[2], w2[3]);
+        *reinterpret_cast<uint2*>(p.w2h + (size_t)u * HID * D + o2) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&f01), *reinterpret_cast<const uint32_t*>(&f23));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tile[rr][4 * c + i] = g1[i];  // gW1^T[h][d]
     }
     __syncthreads();
-    for (int dd = ty; dd < 64; dd += 4) {  // W1*[d][h0 + tx]
-        const size_t idx = (size_t)dd * HID + h0 + tx;
-        const float w1 = p.w1[(size_t)hd * D * HID + idx] - p.eta_over_n * tile[tx][dd];
-        if (p.w1_star) p.w1_star[(size_t)u * D * HID + idx] = w1;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
-        p.w1b[(size_t)u * 2 * D * HID + idx] = hi;
-        p.w1b[(size_t)u * 2 * D * HID + D * HID + idx] = __float2bfloat16_rn(w1 - __bfloat162float(hi));
+    for (int dd = ty; dd < 64; dd += 16) {  // W1*[d][h0 + 4 c .. h0 + 4 c + 3]
+        const size_t idx = (size_t)dd * HID + h0 + 4 * c;
+        const float4 w1o = *reinterpret_cast<const float4*>(p.w1 + (size_t)hd * D * HID + idx);
+        const float w1[4] = {w1o.x - p.eta_over_n * tile[4 * c][dd], w1o.y - p.eta_over_n * tile[4 * c + 1][dd],
+                             w1o.z - p.eta_over_n * tile[4 * c + 2][dd], w1o.w - p.eta_over_n * tile[4 * c + 3][dd]};
+        if (p.w1_star)
+            *reinterpret_cast<float4*>(p.w1_star + (size_t)u * D * HID + idx) = make_float4(w1[0], w1[1], w1[2], w1[3]);
+        uint32_t hi[2], lo[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const __nv_bfloat16 h0b = __float2bfloat16_rn(w1[2 * j]), h1b = __float2bfloat16_rn(w1[2 * j + 1]);
+            const __nv_bfloat16 l0b = __float2bfloat16_rn(w1[2 * j] - __bfloat162float(h0b));
+            const __nv_bfloat16 l1b = __float2bfloat16_rn(w1[2 * j + 1] - __bfloat162float(h1b));
+            hi[j] = (uint32_t)__bfloat16_as_ushort(h0b) | ((uint32_t)__bfloat16_as_ushort(h1b) << 16);
+            lo[j] = (uint32_t)__bfloat16_as_ushort(l0b) | ((uint32_t)__bfloat16_as_ushort(l1b) << 16);
+        }
+        *reinterpret_cast<uint2*>(p.w1b + (size_t)u * 2 * D * HID + idx) = make_uint2(hi[0], hi[1]);
+        *reinterpret_cast<uint2*>(p.w1b + (size_t)u * 2 * D * HID + D * HID + idx) = make_uint2(lo[0], lo[1]);
     }
 }
 
